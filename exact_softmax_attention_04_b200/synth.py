@@ -1,0 +1,150 @@
+"""Seeded synthetic inputs and workload descriptions.
+
+This module is shared by the tests, the benchmark and the smoke check. It
+draws random numbers and names workloads; it does none of the attention
+arithmetic, so both the CUDA path and the CPU oracle can take their inputs
+from here without sharing any computation.
+
+Recipe (stated once, used everywhere): a CPU ``torch.Generator`` seeded with
+``seed`` draws Q, then K, then V, each as fp32 standard normals of shape
+[B, H, n, d]; Q is multiplied by ``q_std``; each tensor is then rounded to
+bf16 (round to nearest even). Layout is contiguous [B, H, n, d], the
+(batch, heads, tokens, head size) order of the naive-versus-fused timing
+snippet on "Efficient Transformers: Sparse Attention, Linear Attention and
+FlashAttention" (section "Family 3").
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional, Tuple
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, mask and input distribution."""
+
+    name: str
+    B: int
+    H: int
+    n: int
+    d: int
+    causal: bool
+    window: int = -1  # < 0: no window; >= 0: keys max(0, i - window) .. i
+    q_std: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def mask(self) -> str:
+        if self.window >= 0:
+            return f"window{self.window}"
+        return "causal" if self.causal else "none"
+
+    def describe(self) -> dict:
+        return {
+            "workload": self.name,
+            "B": self.B,
+            "H": self.H,
+            "n": self.n,
+            "d": self.d,
+            "mask": self.mask,
+            "scale": f"1/sqrt({self.d})",
+            "q_std": self.q_std,
+            "seed": self.seed,
+        }
+
+
+def attended_pairs_per_head(n: int, causal: bool, window: int) -> int:
+    """Number of (query, key) pairs a mask allows in one head.
+
+    none: n*n; causal: n(n+1)/2; causal window w: sum over i of
+    min(i, w) + 1. Used only to count the unmasked FLOPs (4*d per pair).
+    """
+    if window >= 0:
+        w = window
+        if w >= n - 1:
+            return n * (n + 1) // 2
+        # rows 0..w attend i+1 keys, rows w+1..n-1 attend w+1 keys
+        return (w + 1) * (w + 2) // 2 + (n - w - 1) * (w + 1)
+    if causal:
+        return n * (n + 1) // 2
+    return n * n
+
+
+def unmasked_flops(wl: Workload) -> int:
+    """4*d FLOPs per attended pair (2*d for QK^T, 2*d for PV), times B*H."""
+    return 4 * wl.d * attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H
+
+
+def make_qkv(B: int, H: int, n: int, d: int, seed: int = 0, q_std: float = 1.0
+             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Q, K, V as contiguous bf16 CPU tensors [B, H, n, d] (recipe above)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, H, n, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q.mul_(q_std)
+    q = q.to(torch.bfloat16)
+    k = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return q.contiguous(), k.contiguous(), v.contiguous()
+
+
+def make_inputs(wl: Workload):
+    return make_qkv(wl.B, wl.H, wl.n, wl.d, wl.seed, wl.q_std)
+
+
+def sample_rows(B: int, H: int, n: int, per_head_random: int = 256, seed: int = 1,
+                tile: int = 128) -> torch.Tensor:
+    """Deterministic row subset (flat index bh*n + i) for large problems.
+
+    Per head: the first and last 64 rows, the rows on both sides of every
+    8th tile boundary, and ``per_head_random`` uniform rows from a generator
+    seeded with ``seed``. Sorted and unique.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    rows = []
+    edge = list(range(min(64, n))) + list(range(max(0, n - 64), n))
+    bounds = []
+    for b0 in range(tile, n, tile * 8):
+        bounds += [b0 - 1, b0]
+    for bh in range(B * H):
+        r = torch.randint(0, n, (per_head_random,), generator=g).tolist()
+        base = bh * n
+        rows.extend(base + i for i in edge + bounds + r)
+    return torch.unique(torch.tensor(rows, dtype=torch.int64))
+
+
+# The workloads the pages' numbers and the target configurations describe.
+SMALL_CAUSAL = Workload("B1-H2-n256-d64-causal", 1, 2, 256, 64, True)
+FULL_N8192 = Workload("B8-H8-n8192-d64-none", 8, 8, 8192, 64, False)
+WINDOW_N32768 = Workload("B1-H32-n32768-d128-window4096", 1, 32, 32768, 128, True, 4096)
+CAUSAL_N131072 = Workload("B1-H8-n131072-d128-causal", 1, 8, 131072, 128, True)
+
+
+def sweep() -> List[Workload]:
+    """n in {1024, 4096, 16384, 65536} x d in {64, 128} x five masks;
+    B*H*n = 262144 tokens (B=1); Q ~ N(0, 4^2) for large logits."""
+    out = []
+    for n in (1024, 4096, 16384, 65536):
+        for d in (64, 128):
+            H = 262144 // n
+            for causal, window in ((False, -1), (True, -1), (True, 256), (True, 1024), (True, 4096)):
+                m = f"window{window}" if window >= 0 else ("causal" if causal else "none")
+                out.append(Workload(f"sweep-n{n}-d{d}-{m}", 1, H, n, d, causal, window, q_std=4.0))
+    return out
+
+
+def by_name(name: str) -> Optional[Workload]:
+    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072] + sweep():
+        if wl.name == name:
+            return wl
+    return None

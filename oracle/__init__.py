@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for exact softmax attention (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package. The CUDA product path never does.
+
+``attn_oracle.c`` holds the arithmetic; this module compiles it with gcc
+(``build()``) and calls it through ctypes. Inputs are bf16 CPU tensors
+[B, H, n, d]; outputs are fp64 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+KERNEL_SOFTMAX = 0
+KERNEL_IDENTITY = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        i64, dbl, vp, ip = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
+        lib.oracle_attn_rows_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, ip,
+                                             vp, i64, vp, vp, vp]
+        lib.oracle_attn_rows_f64.restype = ip
+        lib.oracle_attn_fwd_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, vp, vp]
+        lib.oracle_attn_fwd_f64.restype = ip
+        lib.oracle_matmul_f64.argtypes = [i64, i64, i64, vp, ip, vp, ip, vp]
+        lib.oracle_matmul_f64.restype = ip
+        lib.oracle_mask_row.argtypes = [i64, i64, ip, i64, vp]
+        lib.oracle_mask_row.restype = ip
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ip
+        _lib = lib
+    return _lib
+
+
+def _bits(t) -> np.ndarray:
+    """bf16 torch tensor -> contiguous uint16 numpy view of its bit patterns."""
+    import torch
+    if t.dtype != torch.bfloat16:
+        raise TypeError("oracle inputs must be bf16")
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
+              kernel: int = KERNEL_SOFTMAX, want_weights: bool = False
+              ) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
+    """O (nrows x d), LSE (nrows) and optionally weights (nrows x n) for flat rows."""
+    lib = _load()
+    B, H, n, d = q.shape
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.empty((rows.size, d), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    w = np.empty((rows.size, n), dtype=np.float64) if want_weights else None
+    rc = lib.oracle_attn_rows_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, n, d,
+                                  float(scale), int(bool(causal)), int(window), int(kernel),
+                                  rows.ctypes.data, rows.size, o.ctypes.data, lse.ctypes.data,
+                                  w.ctypes.data if w is not None else None)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_rows_f64 rejected its arguments (rc={rc})")
+    return o, lse, w
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1
+             ) -> Tuple[np.ndarray, np.ndarray]:
+    """Full O [B,H,n,d] and LSE [B,H,n] in fp64."""
+    lib = _load()
+    B, H, n, d = q.shape
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    o = np.empty((B, H, n, d), dtype=np.float64)
+    lse = np.empty((B, H, n), dtype=np.float64)
+    rc = lib.oracle_attn_fwd_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, n, d,
+                                 float(scale), int(bool(causal)), int(window),
+                                 o.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_f64 rejected its arguments (rc={rc})")
+    return o, lse
+
+
+def matmul(a: np.ndarray, b: np.ndarray, ta: bool = False, tb: bool = False) -> np.ndarray:
+    """op(a) @ op(b) in fp64 through the oracle's own contraction routine."""
+    lib = _load()
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    b = np.ascontiguousarray(b, dtype=np.float64)
+    m, k = (a.shape[1], a.shape[0]) if ta else a.shape
+    k2, n = (b.shape[1], b.shape[0]) if tb else b.shape
+    if k != k2:
+        raise ValueError("inner dimensions differ")
+    c = np.empty((m, n), dtype=np.float64)
+    rc = lib.oracle_matmul_f64(m, n, k, a.ctypes.data, int(ta), b.ctypes.data, int(tb),
+                               c.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_matmul_f64 rejected its arguments")
+    return c
+
+
+def mask_row(n: int, i: int, causal: bool, window: int) -> np.ndarray:
+    lib = _load()
+    out = np.empty(n, dtype=np.uint8)
+    if lib.oracle_mask_row(n, i, int(bool(causal)), int(window), out.ctypes.data) != 0:
+        raise ValueError("bad mask arguments")
+    return out.astype(bool)
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()

@@ -1,0 +1,244 @@
+/*
+ * Exact scaled dot-product attention, forward pass: the fp64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the checker of the CUDA path, not
+ * part of it. Only the test suite, the smoke check and the benchmark's CPU
+ * baseline may load it. It shares no code, header, table or helper with the
+ * CUDA library, and the CUDA library never calls it.
+ *
+ * What it computes is the plain definition, written out:
+ *
+ *   Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V
+ *     ("week17 efficiency attention", recall of scaled dot-product attention;
+ *      "Quadratic cost and efficient attention", section "Where the n^2 hides")
+ *
+ * with the row softmax taken only over the keys a mask allows. For query row
+ * i the allowed key set A(i) is
+ *   none   : every key j < n
+ *   causal : j <= i  (the triu(..., 1) mask of naive_attention in
+ *            "Efficient Transformers ...", section "Family 3")
+ *   window : max(0, i - w) <= j <= i  (the causal sliding-window mask code on
+ *            "week17 efficiency attention", section on local attention)
+ * Then, all in fp64 over the bf16-decoded inputs,
+ *   s_ij  = scale * sum_c q_ic k_jc          for j in A(i)
+ *   M_i   = max_{j in A(i)} s_ij
+ *   Z_i   = sum_{j in A(i)} exp(s_ij - M_i)
+ *   O_i   = sum_{j in A(i)} exp(s_ij - M_i) v_j / Z_i
+ *   LSE_i = M_i + ln Z_i        (natural-log units)
+ *
+ * It is a two-pass softmax over an explicit per-row mask vector; it never
+ * forms the n x n matrix, so a single row of any size can be checked.
+ * There is no tiling, no online rescaling and no reordering beyond the
+ * definition. OpenMP spreads independent rows over host cores.
+ *
+ * The "identity" kernel (ORACLE_KERNEL_IDENTITY) replaces the softmax weight
+ * exp(s_ij - M_i)/Z_i by the raw score s_ij and uses no mask: it yields the
+ * unnormalised product (Q K^T) V * scale, which the associativity identity
+ * (Q K^T) V = Q (K^T V) on "Sparse & sub-quadratic attention" (section
+ * "Escape 2 - change the operator") pins from outside.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_KERNEL_SOFTMAX 0
+#define ORACLE_KERNEL_IDENTITY 1
+
+/* bf16 is the upper half of an IEEE binary32: widen exactly, then to fp64. */
+static double bf16_to_f64(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* sum_c a[c*sa] * b[c*sb], c = 0 .. len-1, in order. */
+double oracle_dot_f64(const double *a, int64_t sa, const double *b, int64_t sb, int64_t len)
+{
+    double acc = 0.0;
+    for (int64_t c = 0; c < len; ++c)
+        acc += a[c * sa] * b[c * sb];
+    return acc;
+}
+
+/*
+ * C[m x n] = op(A) op(B), row-major, op(X) = X or X^T.
+ * A is stored m x k (ta = 0) or k x m (ta = 1); B is stored k x n (tb = 0)
+ * or n x k (tb = 1). Built from oracle_dot_f64 so that the contraction used
+ * by the attention rows is the one the associativity test exercises.
+ */
+int oracle_matmul_f64(int64_t m, int64_t n, int64_t k, const double *A, int ta,
+                      const double *B, int tb, double *C)
+{
+    if (m < 0 || n < 0 || k < 0 || (!A && m * k) || (!B && k * n) || (!C && m * n))
+        return 1;
+    for (int64_t i = 0; i < m; ++i) {
+        const double *arow = ta ? A + i : A + i * k;
+        int64_t sa = ta ? m : 1;
+        for (int64_t j = 0; j < n; ++j) {
+            const double *bcol = tb ? B + j * k : B + j;
+            int64_t sb = tb ? 1 : n;
+            C[i * n + j] = oracle_dot_f64(arow, sa, bcol, sb, k);
+        }
+    }
+    return 0;
+}
+
+/* Explicit mask row: allowed[j] = 1 iff key j is in A(i). */
+int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned char *allowed)
+{
+    if (n < 0 || i < 0 || i >= n || !allowed)
+        return 1;
+    for (int64_t j = 0; j < n; ++j) {
+        int ok = 1;
+        if (causal && j > i)
+            ok = 0;
+        if (window >= 0 && j < i - window)
+            ok = 0;
+        allowed[j] = (unsigned char)ok;
+    }
+    return 0;
+}
+
+/*
+ * Attention for a list of rows.
+ *   q, k, v : bf16 bit patterns, contiguous [B, H, n, d]
+ *   rows    : flat row ids r = (b*H + h)*n + i, nrows of them
+ *   o       : nrows x d   fp64 output (row-major, in the order of rows)
+ *   lse     : nrows       fp64 output (may be NULL)
+ *   weights : nrows x n   fp64 normalised weights, 0 where masked (may be NULL)
+ *   kernel  : ORACLE_KERNEL_SOFTMAX or ORACLE_KERNEL_IDENTITY
+ * window >= 0 requires causal. Returns 0 on success, nonzero on bad input.
+ */
+int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int64_t B, int64_t H, int64_t n, int64_t d, double scale,
+                         int causal, int64_t window, int kernel,
+                         const int64_t *rows, int64_t nrows,
+                         double *o, double *lse, double *weights)
+{
+    if (!q || !k || !v || !o || (!rows && nrows) || B <= 0 || H <= 0 || n <= 0 || d <= 0)
+        return 1;
+    if (window >= 0 && !causal)
+        return 1;
+    if (kernel != ORACLE_KERNEL_SOFTMAX && kernel != ORACLE_KERNEL_IDENTITY)
+        return 1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= B * H * n)
+            return 1;
+
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+        double *kj = (double *)malloc(sizeof(double) * (size_t)d);
+        double *s = (double *)malloc(sizeof(double) * (size_t)n);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        unsigned char *allowed = (unsigned char *)malloc((size_t)n);
+        if (!qi || !kj || !s || !acc || !allowed) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t bh = rows[r] / n;
+                int64_t i = rows[r] % n;
+                const uint16_t *Kh = k + bh * n * d;
+                const uint16_t *Vh = v + bh * n * d;
+                for (int64_t c = 0; c < d; ++c)
+                    qi[c] = bf16_to_f64(q[(bh * n + i) * d + c]);
+
+                if (kernel == ORACLE_KERNEL_IDENTITY) {
+                    for (int64_t j = 0; j < n; ++j)
+                        allowed[j] = 1;
+                } else {
+                    oracle_mask_row(n, i, causal, window, allowed);
+                }
+
+                /* pass 1: scores of allowed keys and their maximum */
+                double M = -INFINITY;
+                for (int64_t j = 0; j < n; ++j) {
+                    if (!allowed[j]) {
+                        s[j] = -INFINITY;
+                        continue;
+                    }
+                    for (int64_t c = 0; c < d; ++c)
+                        kj[c] = bf16_to_f64(Kh[j * d + c]);
+                    s[j] = scale * oracle_dot_f64(qi, 1, kj, 1, d);
+                    if (s[j] > M)
+                        M = s[j];
+                }
+
+                /* pass 2: weights, normaliser and weighted sum of values */
+                for (int64_t c = 0; c < d; ++c)
+                    acc[c] = 0.0;
+                double Z = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    if (!allowed[j])
+                        continue;
+                    double w = (kernel == ORACLE_KERNEL_IDENTITY) ? s[j] : exp(s[j] - M);
+                    Z += w;
+                    for (int64_t c = 0; c < d; ++c)
+                        acc[c] += w * bf16_to_f64(Vh[j * d + c]);
+                }
+
+                if (kernel == ORACLE_KERNEL_IDENTITY) {
+                    for (int64_t c = 0; c < d; ++c)
+                        o[r * d + c] = acc[c];
+                    if (lse)
+                        lse[r] = NAN;
+                    if (weights)
+                        for (int64_t j = 0; j < n; ++j)
+                            weights[r * n + j] = s[j];
+                } else {
+                    for (int64_t c = 0; c < d; ++c)
+                        o[r * d + c] = acc[c] / Z;
+                    if (lse)
+                        lse[r] = M + log(Z);
+                    if (weights)
+                        for (int64_t j = 0; j < n; ++j)
+                            weights[r * n + j] = allowed[j] ? exp(s[j] - M) / Z : 0.0;
+                }
+            }
+        }
+        free(qi);
+        free(kj);
+        free(s);
+        free(acc);
+        free(allowed);
+    }
+    return bad ? 2 : 0;
+}
+
+/* Every row of every head: o is [B, H, n, d] fp64, lse is [B, H, n] fp64. */
+int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        int64_t B, int64_t H, int64_t n, int64_t d, double scale,
+                        int causal, int64_t window, double *o, double *lse)
+{
+    if (B <= 0 || H <= 0 || n <= 0)
+        return 1;
+    int64_t total = B * H * n;
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)total);
+    if (!rows)
+        return 2;
+    for (int64_t r = 0; r < total; ++r)
+        rows[r] = r;
+    int rc = oracle_attn_rows_f64(q, k, v, B, H, n, d, scale, causal, window,
+                                  ORACLE_KERNEL_SOFTMAX, rows, total, o, lse, NULL);
+    free(rows);
+    return rc;
+}
+
+/* Threads an OpenMP parallel region of this library uses. */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
