@@ -1,0 +1,384 @@
+"""Benchmark: attention forward TFLOP/s (unmasked FLOPs) on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload NAME]
+
+One step = one attention forward (the whole hot path: one kernel launch) over
+the workload B=8, H=8, n=8192, d=64, no mask, bf16 Q/K/V ~ N(0,1) from seed 0
+(the 8x8x8192 worked example of "Quadratic cost and efficient attention",
+d_model 512 over 8 heads). FLOPs counted: 4*d per attended (query, key) pair.
+Inputs (201 MB) and outputs exceed the 126 MB L2, so no explicit flush is
+done between steps. Under torchrun every rank runs its own replica (the work
+shards by (batch, head) with no exchange), so scaling is weak and the value is
+the sum of all ranks' FLOPs over the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle on a bounded row sample of the
+same workload (rank 0 only): the deliberately slow reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (unmasked FLOPs) and % of B200 dense BF16 peak"
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_NAME = "attn_fwd_kernel"
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_softmax_attention_04_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"{KERNEL_NAME}.{workload}.traffic.txt")
+    try:
+        vals = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("kernel_sources_sha256_16") != kernel_source_hash():
+            return None
+        return int(vals["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local = _env_int("LOCAL_RANK", 0)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline_leg(wl, o_gpu=None, lse_gpu=None, target_s: float = 15.0):
+    """Oracle timed on this host's cores over a bounded row sample of the
+    workload; also compares those rows with the GPU outputs if given."""
+    import numpy as np
+    import oracle
+    from exact_softmax_attention_04_b200 import synth
+    oracle.build()
+    q, k, v = synth.make_inputs(wl)
+    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window)
+    flops_per_row = 4.0 * wl.d * pairs / wl.n
+    g = torch.Generator().manual_seed(2)
+    total = wl.B * wl.H * wl.n
+    # calibrate on a small sample, then size the sample to ~target_s seconds
+    probe = torch.randint(0, total, (64,), generator=g).numpy()
+    t0 = time.perf_counter()
+    oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    nrows = int(min(total, max(64, 64 * target_s / dt)))
+    rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
+    t0 = time.perf_counter()
+    o_ref, lse_ref, _ = oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, rows)
+    dt = time.perf_counter() - t0
+    out = {"value": nrows * flops_per_row / dt / 1e12, "unit": "TFLOP/s",
+           "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{nrows} random query rows (seed 2) of {wl.name}, fp64 two-pass softmax, "
+                     f"{dt:.1f} s wall",
+           "seconds": dt}
+    if o_gpu is not None:
+        idx = torch.as_tensor(rows, device=o_gpu.device)
+        og = o_gpu.view(-1, wl.d)[idx].float().cpu().numpy()
+        lg = lse_gpu.view(-1)[idx].cpu().numpy()
+        diff = og - o_ref
+        out["parity_vs_gpu"] = {
+            "rows": int(nrows),
+            "o_max_abs": float(np.abs(diff).max()),
+            "o_rel_rms": float(np.sqrt((diff ** 2).sum() / (o_ref ** 2).sum())),
+            "lse_max_abs": float(np.abs(lg - lse_ref).max()),
+        }
+    return out
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    from exact_softmax_attention_04_b200 import synth
+    oracle.build()
+    q, k, v = synth.make_inputs(wl)
+    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window)
+    flops_per_row = 4.0 * wl.d * pairs / wl.n
+    total = wl.B * wl.H * wl.n
+    g = torch.Generator().manual_seed(3)
+    # each step: a bounded sample sized so warmup + steps stay within ~2 minutes
+    probe = torch.randint(0, total, (32,), generator=g).numpy()
+    t0 = time.perf_counter()
+    oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    per_row = max((time.perf_counter() - t0) / 32, 1e-6)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nrows = int(max(8, min(total, budget / per_row)))
+    samples = [np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
+               for _ in range(args.steps + args.warmup)]
+    for i in range(args.warmup):
+        oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, samples[i])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, samples[args.warmup + i])
+    dt = time.perf_counter() - t0
+    value = args.steps * nrows * flops_per_row / dt / 1e12
+    sample = f"{nrows} random query rows per step (seed 3) of {wl.name}, fp64 oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**wl.describe(), "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, wl, world, rank, local):
+    import exact_softmax_attention_04_b200 as attn
+    from exact_softmax_attention_04_b200 import synth
+
+    dev = torch.device("cuda", local)
+    q, k, v = synth.make_inputs(wl)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = synth.unmasked_flops(wl)
+
+    def step():
+        attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start_all = torch.cuda.Event(enable_timing=True)
+        end_all = torch.cuda.Event(enable_timing=True)
+        start_all.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        end_all.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    total_ms = max_over_ranks(start_all.elapsed_time(end_all), world)
+    per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+
+    # end to end through the host-buffer entry point: H2D of q,k,v, kernel,
+    # D2H of o and lse, every step
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    lh = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
+           "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
+    attn.host_staging_release()
+
+    bf16_peak, hbm_peak, peak_src = peaks()
+    achieved = flops / (per_launch_ms / 1e3) / 1e12
+    traffic = recorded_traffic(wl.name)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "algorithmic_flops_per_launch": flops,
+                "min_hbm_bytes_per_launch": 4 * q.numel() * 2 + lse.numel() * 4,
+                "kernel_ms_per_launch": per_launch_ms}
+    if traffic is not None:
+        roofline["traffic_gbs"] = traffic / (per_launch_ms / 1e3) / 1e9
+
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**wl.describe(), "global_batch": wl.B * world, "seq_len": wl.n,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "no flush: inputs 201 MB + outputs 69 MB per step exceed the 126 MB L2"},
+        "pct_of_peak": 100.0 * value / world / bf16_peak,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(wl, o, lse, target_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="B8-H8-n8192-d64-none")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from exact_softmax_attention_04_b200 import synth
+    wl = synth.by_name(args.workload)
+    if wl is None:
+        raise SystemExit(f"unknown workload {args.workload}")
+    if args.impl == "reference":
+        # CPU-only arm: no process group; under torchrun only rank 0 works.
+        return run_reference(args, wl, _env_int("WORLD_SIZE", 1), _env_int("RANK", 0))
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        return run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,170 @@
+"""Exact softmax attention forward for B200 (sm_100a): Python binding.
+
+Argument marshalling only. Every step of the computation runs in the CUDA
+kernels of ``libattn_b200.so`` (built in-tree by ``build_lib.py``); this module
+checks tensor properties, allocates outputs with torch and passes raw
+pointers and the current CUDA stream through the C ABI of ``include/attn.h``.
+There is no CPU fallback: the first call that needs the library raises if
+it is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+
+# Every symbol include/attn.h declares.
+EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_host_staging_release", "attn_sync_status",
+           "attn_strerror", "attn_attended_pairs")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (status {code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m exact_softmax_attention_04_b200.build_lib` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64
+    fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd.argtypes = fwd_args
+    lib.attn_fwd.restype = i
+    lib.attn_fwd_host.argtypes = fwd_args
+    lib.attn_fwd_host.restype = i
+    lib.attn_host_staging_release.argtypes = []
+    lib.attn_host_staging_release.restype = i
+    lib.attn_sync_status.argtypes = [vp]
+    lib.attn_sync_status.restype = i
+    lib.attn_strerror.argtypes = [i]
+    lib.attn_strerror.restype = ctypes.c_char_p
+    lib.attn_attended_pairs.argtypes = [i64, i, i64]
+    lib.attn_attended_pairs.restype = i64
+    return lib
+
+
+_lib_handle: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libattn_b200.so (loaded on first use)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+def strerror(code: int) -> str:
+    return lib().attn_strerror(int(code)).decode()
+
+
+def attended_pairs(n: int, causal: bool, window: int = -1) -> int:
+    r = lib().attn_attended_pairs(int(n), int(bool(causal)), int(window))
+    if r < 0:
+        raise ValueError("bad mask arguments")
+    return int(r)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device: bool) -> None:
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bf16")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, n, d]")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if device and not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not device and t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k and v must have the same shape")
+    if device and not (q.device == k.device == v.device):
+        raise ValueError("q, k and v must be on one device")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+             causal: bool = False, window: int = -1, out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O = softmax(scale * Q K^T) V and its per-row log-sum-exp, on the GPU.
+
+    q, k, v: bf16 CUDA tensors [B, H, n, d], contiguous, d in {64, 128}.
+    causal / window: see include/attn.h (window >= 0 needs causal).
+    Returns (o bf16 [B, H, n, d], lse fp32 [B, H, n]); enqueued on ``stream``
+    (default: the current stream), asynchronous like any CUDA op.
+    """
+    _check_qkv(q, k, v, device=True)
+    B, H, n, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (B, H, n) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, n]")
+    with torch.cuda.device(q.device):
+        rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                           B, H, n, d, float(scale), int(bool(causal)), int(window),
+                           _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+                  causal: bool = False, window: int = -1, out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                  device: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The same operation on host (ideally pinned) tensors: the library copies
+    q, k, v to the device, runs the kernel and copies o and lse back, all on
+    ``stream``. Synchronize the stream before reading the outputs."""
+    _check_qkv(q, k, v, device=False)
+    B, H, n, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    pin = q.is_pinned()
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=pin)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, pin_memory=pin)
+    with torch.cuda.device(device):
+        rc = lib().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, H, n, d, float(scale), int(bool(causal)),
+                                int(window), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_host")
+    return out, lse
+
+
+def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronize ``stream`` and return (and clear) the device status."""
+    return int(lib().attn_sync_status(_stream_handle(stream)))
+
+
+def host_staging_release() -> int:
+    return int(lib().attn_host_staging_release())

@@ -1,0 +1,255 @@
+// attn_api.cu - host side of libattn_b200.so: argument checks, TMA descriptor
+// encoding, launch, device status word, host-buffer entry point.
+// The C declarations and their contracts are in include/attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+bool g_encode_tried = false;
+int *g_status[kMaxDevices] = {};
+bool g_smem_set[kMaxDevices][2] = {};
+
+struct Staging {
+    void *buf = nullptr;
+    size_t cap = 0;
+};
+Staging g_staging[kMaxDevices];
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode_tried) {
+        g_encode_tried = true;
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    return g_encode;
+}
+
+// Device status word for the current device, allocated once and zeroed.
+int *status_word(int dev)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status[dev]) {
+        int *p = nullptr;
+        if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) return nullptr;
+        if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) {
+            cudaFree(p);
+            return nullptr;
+        }
+        g_status[dev] = p;
+    }
+    return g_status[dev];
+}
+
+// [B*H, n, d] bf16 viewed as a 3-D tensor (d fastest), boxes of 64 x 128 x 1,
+// 128-byte swizzle; rows past n read as zero and are clipped on store.
+bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int64_t bh,
+                 int64_t n, int64_t d)
+{
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                          static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(n * d * 2)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(attn_sm100::BOX_COLS),
+                         static_cast<cuuint32_t>(attn_sm100::BM), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_args(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
+               int H, int n, int d, float scale, int causal, int window, bool device_buffers)
+{
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+    if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    if (bh > INT_MAX) return ATTN_ERR_INVALID;
+    if (bh * n > INT64_MAX / (2 * static_cast<int64_t>(d))) return ATTN_ERR_INVALID;
+    if (device_buffers && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+                           !aligned(o, 16) || !aligned(lse, 4)))
+        return ATTN_ERR_INVALID;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (window >= 0 && !causal) return ATTN_ERR_UNSUPPORTED;
+    if (n > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
+    const int64_t tiles = bh * ((n + attn_sm100::BM - 1) / attn_sm100::BM);
+    if (tiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+template <int D>
+int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int n,
+               float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+{
+    using Cfg = attn_sm100::FwdCfg<D>;
+    auto enc = encoder();
+    if (!enc) return ATTN_ERR_CUDA;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
+        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mo, o, bh, n, D))
+        return ATTN_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = g_smem_set[dev][D == 128 ? 1 : 0];
+        if (!set) {
+            if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM_BYTES) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            set = true;
+        }
+    }
+    attn_sm100::FwdParams p;
+    p.lse = lse;
+    p.status = status;
+    p.n = n;
+    p.num_q_tiles = (n + attn_sm100::BM - 1) / attn_sm100::BM;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal;
+    p.window = window < 0 ? -1 : window;
+    const unsigned grid = static_cast<unsigned>(bh * p.num_q_tiles);
+    attn_sm100::attn_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                        int H, int n, int d, float scale, int causal, int window, void *stream)
+{
+    const int rc = check_args(q, k, v, o, lse, B, H, n, d, scale, causal, window, true);
+    if (rc != ATTN_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    int *status = status_word(dev);
+    if (!status) return ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status);
+    return launch_fwd<128>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status);
+}
+
+extern "C" int attn_fwd_host(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                             int H, int n, int d, float scale, int causal, int window, void *stream)
+{
+    int rc = check_args(q, k, v, o, lse, B, H, n, d, scale, causal, window, false);
+    if (rc != ATTN_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    const size_t elems = static_cast<size_t>(B) * H * n * d;
+    const size_t tb = (elems * 2 + 255) & ~static_cast<size_t>(255);
+    const size_t lb = (static_cast<size_t>(B) * H * n * 4 + 255) & ~static_cast<size_t>(255);
+    const size_t need = 4 * tb + lb;
+    char *buf = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        Staging &s = g_staging[dev];
+        if (s.cap < need) {
+            if (s.buf) {
+                cudaDeviceSynchronize();
+                cudaFree(s.buf);
+                s.buf = nullptr;
+                s.cap = 0;
+            }
+            if (cudaMalloc(&s.buf, need) != cudaSuccess) {
+                s.buf = nullptr;
+                return ATTN_ERR_CUDA;
+            }
+            s.cap = need;
+        }
+        buf = static_cast<char *>(s.buf);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *dq = buf, *dk = buf + tb, *dv = buf + 2 * tb, *dout = buf + 3 * tb;
+    float *dl = reinterpret_cast<float *>(buf + 4 * tb);
+    if (cudaMemcpyAsync(dq, q, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    rc = attn_fwd(dq, dk, dv, dout, dl, B, H, n, d, scale, causal, window, stream);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o, dout, elems * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(lse, dl, static_cast<size_t>(B) * H * n * 4, cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" int attn_host_staging_release(void)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    Staging &s = g_staging[dev];
+    if (s.buf) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+        if (cudaFree(s.buf) != cudaSuccess) return ATTN_ERR_CUDA;
+        s.buf = nullptr;
+        s.cap = 0;
+    }
+    return ATTN_OK;
+}
+
+extern "C" int attn_sync_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    int *w = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        w = g_status[dev];
+    }
+    if (!w) return ATTN_OK;  // nothing launched on this device yet
+    int h = 0;
+    if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (h != 0) {
+        if (cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+        return ATTN_ERR_TIMEOUT;
+    }
+    return ATTN_OK;
+}
+
+extern "C" const char *attn_strerror(int status)
+{
+    switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head size must be 64 or 128; a window needs causal=1)";
+    case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+    case ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait; outputs are undefined";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int64_t attn_attended_pairs(int64_t n, int causal, int64_t window)
+{
+    if (n < 0 || (window >= 0 && !causal)) return -1;
+    if (window >= 0 && window < n - 1)
+        return (window + 1) * (window + 2) / 2 + (n - window - 1) * (window + 1);
+    if (causal) return n * (n + 1) / 2;
+    return n * n;
+}

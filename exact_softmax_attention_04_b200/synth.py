@@ -102,24 +102,23 @@ def make_inputs(wl: Workload):
 
 
 def sample_rows(B: int, H: int, n: int, per_head_random: int = 256, seed: int = 1,
-                tile: int = 128) -> torch.Tensor:
+                tile: int = 128, bound_every: int = 8, edge: int = 64) -> torch.Tensor:
     """Deterministic row subset (flat index bh*n + i) for large problems.
 
-    Per head: the first and last 64 rows, the rows on both sides of every
-    8th tile boundary, and ``per_head_random`` uniform rows from a generator
-    seeded with ``seed``. Sorted and unique.
+    Per head: the first and last ``edge`` rows, the two rows on both sides of
+    every ``bound_every``-th tile boundary, and ``per_head_random`` uniform rows
+    from a generator seeded with ``seed``. Sorted and unique.
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     rows = []
-    edge = list(range(min(64, n))) + list(range(max(0, n - 64), n))
-    bounds = []
-    for b0 in range(tile, n, tile * 8):
-        bounds += [b0 - 1, b0]
+    fixed = list(range(min(edge, n))) + list(range(max(0, n - edge), n))
+    for b0 in range(tile, n, tile * bound_every):
+        fixed += [b0 - 1, b0]
     for bh in range(B * H):
         r = torch.randint(0, n, (per_head_random,), generator=g).tolist()
         base = bh * n
-        rows.extend(base + i for i in edge + bounds + r)
+        rows.extend(base + i for i in fixed + r)
     return torch.unique(torch.tensor(rows, dtype=torch.int64))
 
 

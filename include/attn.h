@@ -1,0 +1,131 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact softmax attention forward library
+ * (libattn_b200.so).
+ *
+ * The operation (all entry points that compute):
+ *
+ *   O = softmax(scale * Q K^T) V,   row-wise softmax over the allowed keys,
+ *   LSE_i = ln sum_{j allowed for i} exp(scale * q_i . k_j)
+ *
+ * Scaled dot-product attention is defined on "week17 efficiency attention"
+ * (recall at the top of the page: softmax(Q K^T / sqrt(d_k)) V) and on
+ * "Quadratic cost and efficient attention" (section "Where the n^2 hides").
+ * It is computed tile by tile with an online softmax (running row maximum and
+ * normaliser), as described under FlashAttention on "week17 efficiency
+ * attention" and in "The online softmax trick" on "Efficient Transformers:
+ * Sparse Attention, Linear Attention and FlashAttention"; the n x n score
+ * matrix is never written to device memory (same page, "Family 3").
+ *
+ * Masks (key j allowed for query i):
+ *   causal = 0, window < 0  : every j in [0, n)               (no mask)
+ *   causal = 1, window < 0  : j <= i                          (causal; the triu
+ *                              mask of naive_attention, "Family 3")
+ *   causal = 1, window >= 0 : max(0, i - window) <= j <= i    (causal sliding
+ *                              window; the window-mask snippet on "week17
+ *                              efficiency attention", local attention section;
+ *                              min(i, window) + 1 keys including i itself)
+ *   causal = 0, window >= 0 : ATTN_ERR_UNSUPPORTED (the symmetric window
+ *                              i-w .. i+w of the same page is not provided)
+ *
+ * Layout: Q, K, V and O are bf16, contiguous [B, H, n, d] (token-major inside
+ * each head, d fastest). LSE is fp32, contiguous [B, H, n], natural-log units.
+ * Arithmetic: bf16 inputs, fp32 accumulation (QK^T and PV on the tensor
+ * cores), fp32 softmax, P rounded to bf16 before PV, O rounded to bf16 (round
+ * to nearest even).
+ *
+ * Ownership: the caller owns every buffer passed in and keeps it alive until
+ * the work enqueued on `stream` has finished. The library owns only: one
+ * lazily allocated device status word per device, and, for attn_fwd_host, a
+ * per-device set of device staging buffers (grown on demand, released by
+ * attn_host_staging_release). No entry point prints, exits, aborts or traps.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream). Work is enqueued on it on the calling thread's current device; the
+ * device pointers must belong to that device.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stdint.h>
+
+/* Exported symbols of the shared library (everything else is hidden). */
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    ATTN_OK = 0,              /* success (for async calls: enqueued)            */
+    ATTN_ERR_INVALID = 1,     /* a bad argument; nothing was enqueued           */
+    ATTN_ERR_UNSUPPORTED = 2, /* valid but not provided (d not 64/128, ...)     */
+    ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed              */
+    ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (device side)  */
+} attn_status;
+
+/*
+ * attn_fwd - enqueue the attention forward pass on device buffers.
+ *
+ *   q, k, v : device, bf16 [B, H, n, d], 16-byte aligned, read only
+ *   o       : device, bf16 [B, H, n, d], 16-byte aligned, written
+ *   lse     : device, fp32 [B, H, n], 4-byte aligned, written
+ *   B, H, n : >= 1; B*H*n*d must fit in int64 and B*H < 2^31
+ *   d       : head size; 64 or 128 (else ATTN_ERR_UNSUPPORTED)
+ *   scale   : finite and > 0 (the pages' choice is 1/sqrt(d))
+ *   causal, window : the mask, see the table above
+ *   stream  : cudaStream_t as void*
+ *
+ * Returns ATTN_OK once the kernel is enqueued; ATTN_ERR_INVALID /
+ * ATTN_ERR_UNSUPPORTED before touching the device; ATTN_ERR_CUDA if
+ * encoding the TMA descriptors or the launch fails. A device-side timeout
+ * is reported later by attn_sync_status. o and lse must not overlap q, k, v.
+ */
+ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int n, int d, float scale, int causal, int window,
+             void *stream);
+
+/*
+ * attn_fwd_host - the same operation on HOST buffers, copies included.
+ *
+ *   q, k, v : host, bf16 [B, H, n, d] (pinned memory makes the copies async)
+ *   o, lse  : host, written (bf16 [B, H, n, d] and fp32 [B, H, n])
+ *
+ * Enqueues on `stream`: host-to-device copies of q, k, v into library-owned
+ * staging buffers, attn_fwd, and device-to-host copies of o and lse. The
+ * caller synchronizes `stream` (or calls attn_sync_status) before reading o
+ * and lse. Staging buffers are per device and shared by all calls: calls on
+ * different streams of one device must not overlap. Returns as attn_fwd, or
+ * ATTN_ERR_CUDA if growing the staging buffers fails.
+ */
+ATTN_API int attn_fwd_host(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int H, int n, int d, float scale, int causal, int window,
+                  void *stream);
+
+/* Frees this device's attn_fwd_host staging buffers (synchronizes the device). */
+ATTN_API int attn_host_staging_release(void);
+
+/*
+ * attn_sync_status - synchronize `stream`, then read and clear this device's
+ * status word. Returns ATTN_ERR_TIMEOUT if any kernel since the last call gave
+ * up on a bounded wait (its outputs are then undefined), ATTN_ERR_CUDA if the
+ * synchronization reported a CUDA error, else ATTN_OK.
+ */
+ATTN_API int attn_sync_status(void *stream);
+
+/* Static English text for a status code; never NULL. */
+ATTN_API const char *attn_strerror(int status);
+
+/* Number of attended (query, key) pairs in one head for the given mask;
+ * 4*d FLOPs per pair is the unmasked FLOP count. Returns -1 on bad input. */
+ATTN_API int64_t attn_attended_pairs(int64_t n, int causal, int64_t window);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,113 @@
+"""The C ABI boundary, checked without a GPU: the library builds and loads,
+exports every function include/attn.h declares, and rejects bad arguments
+before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def attn():
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    import exact_softmax_attention_04_b200 as pkg
+    return pkg
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    assert "attn_fwd" in names and "attn_sync_status" in names
+    import exact_softmax_attention_04_b200 as pkg
+    assert sorted(pkg.EXPORTS) == names
+
+
+def test_library_exports_every_declared_symbol(attn):
+    out = subprocess.run(["nm", "-D", "--defined-only", attn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\S+)$", out, flags=re.M))
+    for name in _declared_functions():
+        assert name in exported, name
+        assert hasattr(attn.lib(), name)
+    # nothing else leaks out as a C symbol of ours
+    assert not [s for s in exported if s.startswith("attn_") and s not in _declared_functions()]
+
+
+def test_header_compiles_as_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "attn.h"\n'
+                   'int main(void){ const char *(*f)(int) = attn_strerror; (void)f;'
+                   ' return ATTN_OK; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), "-c",
+                    str(src), "-o", str(tmp_path / "t.o")], check=True)
+
+
+def test_strerror_covers_every_status(attn):
+    texts = {attn.strerror(c) for c in range(5)}
+    assert len(texts) == 5
+    assert attn.strerror(99) == "unknown status"
+
+
+def test_attended_pairs_matches_the_workload_counts(attn):
+    from exact_softmax_attention_04_b200 import synth
+    for n in (1, 2, 127, 128, 129, 1000, 131072):
+        for causal, window in [(False, -1), (True, -1), (True, 0), (True, 1), (True, 256), (True, 4096),
+                               (True, 10 ** 6)]:
+            assert attn.attended_pairs(n, causal, window) == synth.attended_pairs_per_head(n, causal, window)
+    with pytest.raises(ValueError):
+        attn.attended_pairs(10, False, 3)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), 1), (dict(lse=0), 1), (dict(B=0), 1), (dict(H=-1), 1), (dict(n=0), 1),
+    (dict(d=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(scale=-1.0), 1),
+    (dict(scale=float("inf")), 1), (dict(causal=2), 1), (dict(q=FAKE + 8), 1), (dict(lse=FAKE + 2), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(causal=0, window=5), 2), (dict(n=(1 << 30) + 1), 2),
+    (dict(B=1 << 16, H=1 << 16), 1),
+])
+def test_attn_fwd_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, n=128, d=64, scale=0.125,
+             causal=1, window=-1, stream=None)
+    a.update(kw)
+    rc = attn.lib().attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["n"],
+                             a["d"], a["scale"], a["causal"], a["window"], a["stream"])
+    assert rc == code
+
+
+def test_host_entry_point_rejects_bad_arguments(attn):
+    rc = attn.lib().attn_fwd_host(None, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, -1, None)
+    assert rc == attn.ATTN_ERR_INVALID
+    rc = attn.lib().attn_fwd_host(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 80, 0.125, 0, -1, None)
+    assert rc == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_python_binding_checks_tensors_before_calling(attn):
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q)  # host tensors on the device entry point
+    with pytest.raises(TypeError):
+        attn.attn_fwd_host(q.float(), q, q)
+    with pytest.raises(ValueError):
+        attn.attn_fwd_host(q, q[..., :32].contiguous(), q)
+
+
+def test_missing_library_fails_loudly(monkeypatch, attn):
+    import exact_softmax_attention_04_b200 as pkg
+    monkeypatch.setattr(pkg, "LIB_PATH", "/nonexistent/libattn_b200.so")
+    with pytest.raises(ImportError):
+        pkg._load()

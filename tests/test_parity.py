@@ -1,0 +1,149 @@
+"""CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Small problems are compared in full; they span several 128-row/128-key tiles
+and ragged tails. Full-size workloads run in the same launch configuration
+the benchmark times and are compared on a deterministic row sample that the
+oracle computes one row at a time, plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_softmax_attention_04_b200 import synth
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def attn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    import exact_softmax_attention_04_b200 as pkg
+    return pkg
+
+
+def _gpu(attn, q, k, v, causal, window, scale=None):
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), scale, causal, window)
+    assert attn.sync_status() == attn.ATTN_OK
+    return o, lse
+
+
+def _full_check(attn, oracle_mod, q, k, v, causal, window, scale=None, what=""):
+    d = q.shape[-1]
+    sc = scale if scale is not None else 1.0 / np.sqrt(d)
+    o, lse = _gpu(attn, q, k, v, causal, window, scale)
+    o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, sc, causal, window)
+    return assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, what)
+
+
+def _sampled_check(attn, oracle_mod, wl, rows, o=None, lse=None):
+    q, k, v = synth.make_inputs(wl)
+    if o is None:
+        o, lse = _gpu(attn, q, k, v, wl.causal, wl.window, wl.scale)
+    o_s = o.view(-1, wl.d)[torch.as_tensor(rows, device=o.device)].float().cpu().numpy()
+    l_s = lse.view(-1)[torch.as_tensor(rows, device=o.device)].cpu().numpy()
+    o_ref, lse_ref, _ = oracle_mod.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, rows)
+    return assert_close(o_s, l_s, o_ref, lse_ref, wl.name), o, lse
+
+
+def test_small_causal_workload_in_full(attn, oracle_mod):
+    wl = synth.SMALL_CAUSAL
+    q, k, v = synth.make_inputs(wl)
+    _full_check(attn, oracle_mod, q, k, v, wl.causal, wl.window, wl.scale, wl.name)
+
+
+MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 127), (True, 128), (True, 129),
+         (True, 300), (True, 100000)]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n", [1, 77, 128, 129, 256, 383, 640])
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_small_shapes_all_masks_in_full(attn, oracle_mod, d, n, causal, window):
+    q_std = 4.0 if (n + d + window) % 2 else 1.0
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=n * 7 + d, q_std=q_std)
+    _full_check(attn, oracle_mod, q, k, v, causal, window, what=f"n{n} d{d} c{causal} w{window}")
+
+
+def test_batch_and_many_heads(attn, oracle_mod):
+    q, k, v = synth.make_qkv(3, 5, 200, 64, seed=21)
+    for causal, window in [(False, -1), (True, -1), (True, 50)]:
+        _full_check(attn, oracle_mod, q, k, v, causal, window, what=f"B3H5 c{causal} w{window}")
+
+
+def test_non_default_scale(attn, oracle_mod):
+    q, k, v = synth.make_qkv(1, 2, 300, 128, seed=22)
+    for scale in (0.01, 0.3):
+        _full_check(attn, oracle_mod, q, k, v, True, -1, scale=scale, what=f"scale {scale}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_zero_queries_give_mean_of_allowed_values(attn, d):
+    n = 333
+    _, k, v = synth.make_qkv(1, 2, n, d, seed=30)
+    q = torch.zeros_like(k)
+    vf = v.double()
+    for causal, window in [(False, -1), (True, -1), (True, 40)]:
+        o, lse = _gpu(attn, q, k, v, causal, window)
+        o, lse = o.double().cpu(), lse.double().cpu()
+        for i in (0, 1, 39, 40, 41, 127, 128, 200, n - 1):
+            lo = max(0, i - window) if window >= 0 else 0
+            hi = i + 1 if causal else n
+            ref = vf[..., lo:hi, :].mean(dim=-2)
+            assert (o[..., i, :] - ref).abs().max() <= 2e-2
+            assert (lse[..., i] - np.log(hi - lo)).abs().max() <= 1e-3
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_window_zero_returns_values_exactly(attn, d):
+    q, k, v = synth.make_qkv(2, 2, 257, d, seed=31, q_std=4.0)
+    o, lse = _gpu(attn, q, k, v, True, 0)
+    assert torch.equal(o.cpu(), v)
+    ref = (q.double() * k.double()).sum(-1) / np.sqrt(d)
+    assert (lse.double().cpu() - ref).abs().max() <= 1e-3
+
+
+def test_key_value_permutation_invariance(attn):
+    q, k, v = synth.make_qkv(1, 2, 512, 128, seed=32, q_std=4.0)
+    perm = torch.randperm(512, generator=torch.Generator().manual_seed(1))
+    o1, l1 = _gpu(attn, q, k, v, False, -1)
+    o2, l2 = _gpu(attn, q, k[..., perm, :].contiguous(), v[..., perm, :].contiguous(), False, -1)
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    assert (l1 - l2).abs().max().item() <= 1e-3
+
+
+def test_runs_are_deterministic(attn):
+    q, k, v = synth.make_qkv(1, 4, 1000, 64, seed=33)
+    o1, l1 = _gpu(attn, q, k, v, True, 300)
+    o2, l2 = _gpu(attn, q, k, v, True, 300)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_host_entry_point_matches_device_entry_point(attn):
+    q, k, v = synth.make_qkv(2, 3, 700, 128, seed=34)
+    o_d, l_d = _gpu(attn, q, k, v, True, 200)
+    qp, kp, vp = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o_h, l_h = attn.attn_fwd_host(qp, kp, vp, causal=True, window=200)
+    assert attn.sync_status() == attn.ATTN_OK
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+
+
+@pytest.mark.parametrize("wl", synth.sweep(), ids=lambda w: w.name)
+def test_sweep_cells_sampled(attn, oracle_mod, wl):
+    rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=24, bound_every=16)
+    _sampled_check(attn, oracle_mod, wl, rows)
+
+
+@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072],
+                         ids=lambda w: w.name)
+def test_full_size_workloads_sampled(attn, oracle_mod, wl):
+    per_head = 16 if wl.n >= 65536 else 24
+    rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=per_head, bound_every=64, edge=32)
+    _, o, lse = _sampled_check(attn, oracle_mod, wl, rows)
+    assert bool(torch.isfinite(lse).all()) and bool(torch.isfinite(o.float()).all())
+    q, k, v = synth.make_inputs(wl)
+    o2, l2 = _gpu(attn, q, k, v, wl.causal, wl.window, wl.scale)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
