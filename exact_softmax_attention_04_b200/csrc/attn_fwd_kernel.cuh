@@ -42,10 +42,15 @@ constexpr int BOX_BYTES = BM * BOX_COLS * 2; // one [128 x 64] bf16 box: 16 KB
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
 constexpr int STATUS_WAIT_TIMEOUT = 1;
-// Lazy rescaling: keep a stale row max until the new one exceeds it by more
-// than this many log2 units (P entries then stay below 2^8). Exact in real
-// arithmetic because O and l share the same stale max.
-constexpr float RESCALE_THRESHOLD = 8.0f;
+// The running max is replaced as soon as a tile raises it (threshold 0), so
+// the largest P entry of a row is exactly 1.0 and its bf16 rounding never
+// reaches O. A positive threshold (keeping a stale max, P up to 2^threshold)
+// saves O rescales but puts up to 2^-9 relative error on the dominant term,
+// which breaks the 2e-2 max-abs bar on O for peaked rows.
+#ifndef ATTN_RESCALE_THRESHOLD
+#define ATTN_RESCALE_THRESHOLD 0.0f
+#endif
+constexpr float RESCALE_THRESHOLD = ATTN_RESCALE_THRESHOLD;
 
 struct FwdParams {
     float *lse;     // [B*H, n]
