@@ -86,7 +86,7 @@ def recorded_traffic(workload: str):
 class ClockSampler:
     """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -95,6 +95,9 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        self.out = ""
+        if self.gpu < 0:
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
@@ -114,25 +117,30 @@ class ClockSampler:
                 self.proc.kill()
                 self.out, _ = self.proc.communicate()
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and throttle reasons over the samples taken inside
+        [t0, t1] (wall clock, seconds); all samples if none fall inside."""
+        import datetime
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in (self.out or "").splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]),
+                             {nm for nm, val in zip(names, parts[5:9]) if val.lower().startswith("active")}))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        inside = [r for r in rows if t0 is not None and t0 - 0.1 <= r[0] <= t1 + 0.1]
+        use = inside or rows
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set().union(*(r[3] for r in use))
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": use[-1][2],
+                "reasons": sorted(reasons), "samples": len(use),
+                "window": "timed region" if inside else "whole run (no sample inside the timed region)"}
 
 
 def dist_setup(n_gpus: int):
@@ -274,7 +282,10 @@ def run_ours(args, wl, world, rank, local):
           for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local if not args.profile else -1) as clocks:
+        if not args.profile:
+            time.sleep(0.5)  # let the sampler start before the timed region
+        wall0 = time.time()
         start_all = torch.cuda.Event(enable_timing=True)
         end_all = torch.cuda.Event(enable_timing=True)
         start_all.record(stream)
@@ -284,6 +295,7 @@ def run_ours(args, wl, world, rank, local):
             ev[i][1].record(stream)
         end_all.record(stream)
         torch.cuda.synchronize(dev)
+        wall1 = time.time()
     barrier(world)
     st = attn.sync_status(stream)
     if st != attn.ATTN_OK:
@@ -292,6 +304,14 @@ def run_ours(args, wl, world, rank, local):
     per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_per_step = total_ms / args.steps
     value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+
+    bf16_peak, hbm_peak, peak_src = peaks()
+    achieved = flops / (per_launch_ms / 1e3) / 1e12
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": wl.name, "steps": args.steps, "warmup": args.warmup,
+                              "kernel_ms_per_launch": per_launch_ms, "tflops": achieved}), flush=True)
+        return 0
 
     # end to end through the host-buffer entry point: H2D of q,k,v, kernel,
     # D2H of o and lse, every step
@@ -318,8 +338,6 @@ def run_ours(args, wl, world, rank, local):
            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
     attn.host_staging_release()
 
-    bf16_peak, hbm_peak, peak_src = peaks()
-    achieved = flops / (per_launch_ms / 1e3) / 1e12
     traffic = recorded_traffic(wl.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
                 "frac": achieved / bf16_peak, "traffic": traffic,
@@ -339,12 +357,14 @@ def run_ours(args, wl, world, rank, local):
         "data": "synthetic",
         "config": {**wl.describe(), "global_batch": wl.B * world, "seq_len": wl.n,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "no flush: inputs 201 MB + outputs 69 MB per step exceed the 126 MB L2"},
+                   "l2": f"no flush: inputs {3 * q.numel() * 2 / 1e6:.0f} MB + outputs "
+                         f"{(o.numel() * 2 + lse.numel() * 4) / 1e6:.0f} MB per step "
+                         + ("exceed" if 3 * q.numel() * 2 > 126e6 else "do NOT exceed") + " the 126 MB L2"},
         "pct_of_peak": 100.0 * value / world / bf16_peak,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(wall0, wall1),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_leg(wl, o, lse, target_s=args.cpu_seconds)
@@ -355,12 +375,15 @@ def run_ours(args, wl, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="B8-H8-n8192-d64-none")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="timed kernel launches only (no e2e, CPU baseline or clock sampling): "
+                         "the command profiled under ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

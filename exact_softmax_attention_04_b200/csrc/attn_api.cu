@@ -128,10 +128,11 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.status = status;
     p.n = n;
     p.num_q_tiles = (n + attn_sm100::BM - 1) / attn_sm100::BM;
+    p.num_cta_tiles = (p.num_q_tiles + attn_sm100::QT - 1) / attn_sm100::QT;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
     p.window = window < 0 ? -1 : window;
-    const unsigned grid = static_cast<unsigned>(bh * p.num_q_tiles);
+    const unsigned grid = static_cast<unsigned>(bh * p.num_cta_tiles);
     attn_sm100::attn_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -1,32 +1,37 @@
 // attn_fwd_kernel.cuh - exact softmax attention forward for sm_100a.
 //
-// One CTA computes one 128-row query tile Q_i of one (batch, head):
-//   for each key/value tile j allowed by the mask:
-//     S = Q_i K_j^T                       (tcgen05 MMA, smem x smem -> TMEM fp32)
-//     online softmax on S, row by row     (running max m, running normaliser l)
-//     O += P V_j                          (tcgen05 MMA, P from TMEM x V from smem)
-//   O_i = O / l, LSE_i = m + ln l         (written once)
-// This is the FlashAttention tile loop with the online softmax ("week17
-// efficiency attention", FlashAttention section; "Efficient Transformers ...",
-// "The online softmax trick"): the running output is kept unnormalised and
-// divided once at the end, and only the current tile's scores live on chip.
+// One CTA computes two adjacent 128-row query tiles Q_0, Q_1 (256 rows) of
+// one (batch, head). For each key/value tile j allowed by the mask:
+//   S_s = Q_s K_j^T                     (tcgen05 MMA, smem x smem -> TMEM fp32)
+//   online softmax on S_s, row by row   (running max m, running normaliser l)
+//   O_s += P_s V_j                      (tcgen05 MMA, P from TMEM x V from smem)
+// and at the end O_s / l, LSE = m + ln l are written once. This is the
+// FlashAttention tile loop with the online softmax ("week17 efficiency
+// attention", FlashAttention section; "Efficient Transformers ...", "The
+// online softmax trick"): the running output stays unnormalised and is
+// divided once, and only the current tile's scores ever live on chip.
 //
-// Roles (192 threads, 6 warps):
-//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r); reads S,
+// Roles (320 threads, 10 warps):
+//   warps 0-3  softmax for Q_0; warps 4-7 softmax for Q_1. Thread r of a
+//              warpgroup owns query row r (= TMEM lane r): it reads its S row,
 //              masks boundary tiles, updates (m, l), writes P (bf16) back into
-//              TMEM over the S columns, rescales O when the max grew, and runs
-//              the epilogue (O / l -> bf16 -> smem -> TMA store, LSE store).
-//   warp 4     TMA producer (one elected lane): Q once, then K_j and V_j into
-//              an NS-stage shared-memory ring.
-//   warp 5     MMA issuer (one elected lane) and TMEM owner.
-// TMEM columns: S/P double buffer at [0,128) and [128,256), O at [256, 256+D).
-// S_{j+1} is computed while the softmax works on S_j; tcgen05 MMAs issued by
-// one thread execute in order, so S_{j+2} never overwrites P_j before the
-// P_j V_j MMA has read it.
+//              TMEM over its S columns, rescales its O row when m grew, and runs
+//              the epilogue (O / l -> bf16 -> smem -> TMA store; LSE store).
+//   warp 8     MMA issuer (one elected lane) and TMEM owner.
+//   warp 9     TMA producer (one elected lane): Q_0, Q_1 once, then K_j, V_j
+//              alternately into a ring of NSLOT shared-memory slots.
+// TMEM columns: S_0/P_0 [0,128), S_1/P_1 [128,256), O_0 [256, 256+D),
+// O_1 [256+D, 256+2D).
+// MMA issue order per key tile j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j). The
+// two softmax warpgroups thus alternate with the tensor core: while one works
+// on its S, the tensor core runs the other tile's PV and S. tcgen05 MMAs from
+// one thread complete in issue order, so (a) S_s(j) overwrites P_s(j-1) only
+// after PV_s(j-1) has read it, and (b) when S_s(j) is complete, PV_s(j-1) is
+// too, so the softmax may rescale O_s right away.
 //
-// Every wait is bounded (about one second). On expiry the kernel records
-// ATTN device status bit 1, tells the other roles to stop, waits (bounded) for
-// its own copies and MMAs in flight, frees TMEM and returns.
+// Every wait is bounded (about one second). On expiry the kernel sets bit 1
+// of the device status word, tells the other roles to stop, waits (bounded)
+// for its own copies and MMAs in flight, frees TMEM and returns.
 #pragma once
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -35,28 +40,35 @@
 
 namespace attn_sm100 {
 
-constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
-constexpr int BN = 128;  // keys per tile
-constexpr int BOX_COLS = 64;                 // bf16 columns per 128-byte swizzle atom
-constexpr int BOX_BYTES = BM * BOX_COLS * 2; // one [128 x 64] bf16 box: 16 KB
+constexpr int BM = 128;                       // query rows per tile (= TMEM lanes)
+constexpr int BN = 128;                       // keys per tile
+constexpr int QT = 2;                         // query tiles per CTA
+constexpr int BOX_COLS = 64;                  // bf16 columns per 128-byte swizzle atom
+constexpr int BOX_BYTES = BM * BOX_COLS * 2;  // one [128 x 64] bf16 box: 16 KB
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 200000000ull;
 constexpr int STATUS_WAIT_TIMEOUT = 1;
-// The running max is replaced as soon as a tile raises it (threshold 0), so
-// the largest P entry of a row is exactly 1.0 and its bf16 rounding never
-// reaches O. A positive threshold (keeping a stale max, P up to 2^threshold)
-// saves O rescales but puts up to 2^-9 relative error on the dominant term,
-// which breaks the 2e-2 max-abs bar on O for peaked rows.
-#ifndef ATTN_RESCALE_THRESHOLD
-#define ATTN_RESCALE_THRESHOLD 0.0f
+
+// The running max is replaced as soon as a tile raises it, so the largest P
+// entry of every row is exactly 1.0 and its bf16 rounding never reaches O. (A
+// stale max saves O rescales but puts up to 2^-9 relative error on the
+// dominant term: too much for peaked rows.)
+
+// Exponentials computed on the FMA pipe instead of the MUFU unit: out of every
+// 8 pairs of a row chunk, the first ATTN_EX2_EMU pairs use the polynomial.
+#ifndef ATTN_EX2_EMU_D64
+#define ATTN_EX2_EMU_D64 0
 #endif
-constexpr float RESCALE_THRESHOLD = ATTN_RESCALE_THRESHOLD;
+#ifndef ATTN_EX2_EMU_D128
+#define ATTN_EX2_EMU_D128 0
+#endif
 
 struct FwdParams {
-    float *lse;     // [B*H, n]
-    int *status;    // device status word
+    float *lse;        // [B*H, n]
+    int *status;       // device status word
     int n;
-    int num_q_tiles;
+    int num_q_tiles;   // ceil(n / BM)
+    int num_cta_tiles; // ceil(num_q_tiles / QT)
     float scale_log2;  // scale * log2(e)
     int causal;
     int window;        // < 0: none
@@ -65,21 +77,22 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
     static_assert(D == 64 || D == 128, "head size 64 or 128");
-    static constexpr int NS = (D == 128) ? 3 : 4;       // K/V ring depth
-    static constexpr int TILE_BYTES = BM * D * 2;        // 128 rows x D bf16
+    static constexpr int TILE_BYTES = BM * D * 2;    // 128 rows x D bf16
     static constexpr int BOXES = D / BOX_COLS;
+    static constexpr int NSLOT = (D == 128) ? 5 : 8;  // K/V ring slots (one tile each)
     static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + TILE_BYTES;
-    static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
-    static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
-    // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-    // p_full[2], o_done, drain
-    static constexpr int NUM_BARS = 1 + 4 * NS + 2 + 2 + 1 + 1;
+    static constexpr int KV_OFF = Q_OFF + QT * TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // q_full[QT], kv_full[NSLOT], kv_empty[NSLOT], s_full[QT], p_full[QT], o_done[QT], drain
+    static constexpr int NUM_BARS = QT + 2 * NSLOT + 3 * QT + 1;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + 1 KB alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t O_COL = 256;
-    static constexpr int THREADS = 192;
+    static constexpr uint32_t S_COL = 0;    // + s * BN
+    static constexpr uint32_t O_COL = 256;  // + s * D
+    static constexpr int THREADS = 320;
+    static constexpr int EX2_EMU = (D == 128) ? ATTN_EX2_EMU_D128 : ATTN_EX2_EMU_D64;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct Waiter {
@@ -118,12 +131,17 @@ struct Waiter {
     }
 };
 
-// Key tiles [jlo, jhi) that hold at least one key allowed for some row of the
-// query tile starting at m0. Fully masked tiles are never visited.
+// Key tiles [jlo, jhi) holding at least one key allowed for some row of the
+// query tile starting at m0 (fully masked tiles are never visited). Empty when
+// the query tile lies past n.
 __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int window, int &jlo,
                                                int &jhi)
 {
-    const int kend = causal ? min(n, m0 + BM) : n;           // exclusive
+    if (m0 >= n) {
+        jlo = jhi = 0;
+        return;
+    }
+    const int kend = causal ? min(n, m0 + BM) : n;  // exclusive
     const int kbeg = (window >= 0) ? max(0, m0 - window) : 0;
     jlo = kbeg / BN;
     jhi = (kend + BN - 1) / BN;
@@ -132,6 +150,27 @@ __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int wi
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 
+// 2^x on the FMA pipe for x in [-125, 0.5]: x = k + f with k = round(x) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (minimax relative error
+// 7.5e-5, coefficients fitted by gen_exp2_poly.py), 2^k added to the exponent
+// field. Two lanes at a time with packed fp32 instructions.
+__device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float &y0, float &y1)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+    x0 = fmaxf(x0, -125.0f);
+    x1 = fmaxf(x1, -125.0f);
+    const float2 t = fadd2(make_float2(x0, x1), make_float2(kRound, kRound));
+    const float2 r = fadd2(t, make_float2(-kRound, -kRound));        // round(x)
+    const float2 f = fadd2(make_float2(x0, x1), make_float2(-r.x, -r.y));
+    float2 p = ffma2(make_float2(0.05517167f, 0.05517167f), f, make_float2(0.24261113f, 0.24261113f));
+    p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
+    p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
+    // t's low mantissa bits hold k (offset by 0x4B400000, whose bits vanish
+    // when shifted left by 23): add k << 23 to the exponent of p.
+    y0 = u2f(f2u(p.x) + (f2u(t.x) << 23));
+    y1 = u2f(f2u(p.y) + (f2u(t.y) << 23));
+}
+
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -139,66 +178,66 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     const FwdParams p)
 {
     using C = FwdCfg<D>;
-    constexpr int NS = C::NS;
+    constexpr int NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - raw);
 
-    const uint32_t sQ = base + C::Q_OFF;
+    auto sQ = [&](int s) { return base + C::Q_OFF + s * C::TILE_BYTES; };
+    auto sKV = [&](int slot) { return base + C::KV_OFF + slot * C::TILE_BYTES; };
     const uint32_t bars = base + C::BAR_OFF;
-    auto sK = [&](int s) { return base + C::K_OFF + s * C::TILE_BYTES; };
-    auto sV = [&](int s) { return base + C::V_OFF + s * C::TILE_BYTES; };
-    const uint32_t q_full = bars;
-    auto k_full = [&](int s) { return bars + 8u * (1 + s); };
-    auto k_empty = [&](int s) { return bars + 8u * (1 + NS + s); };
-    auto v_full = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
-    auto v_empty = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
-    auto s_full = [&](int b) { return bars + 8u * (1 + 4 * NS + b); };
-    auto p_full = [&](int b) { return bars + 8u * (3 + 4 * NS + b); };
-    const uint32_t o_done = bars + 8u * (5 + 4 * NS);
-    const uint32_t drain_bar = bars + 8u * (6 + 4 * NS);
+    auto q_full = [&](int s) { return bars + 8u * s; };
+    auto kv_full = [&](int slot) { return bars + 8u * (QT + slot); };
+    auto kv_empty = [&](int slot) { return bars + 8u * (QT + NSLOT + slot); };
+    auto s_full = [&](int s) { return bars + 8u * (QT + 2 * NSLOT + s); };
+    auto p_full = [&](int s) { return bars + 8u * (2 * QT + 2 * NSLOT + s); };
+    auto o_done = [&](int s) { return bars + 8u * (3 * QT + 2 * NSLOT + s); };
+    const uint32_t drain_bar = bars + 8u * (4 * QT + 2 * NSLOT);
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
 
-    // Work tile: query tiles of one head are adjacent in blockIdx (K/V reuse in
-    // L2); within a head the late (most expensive under a causal mask) tiles
-    // start first.
-    const int bh = blockIdx.x / p.num_q_tiles;
-    const int qt = p.num_q_tiles - 1 - static_cast<int>(blockIdx.x % p.num_q_tiles);
-    const int m0 = qt * BM;
+    // Work: query-tile pairs of one head are adjacent in blockIdx (K/V reuse in
+    // L2); within a head the late pairs (the most expensive under a causal
+    // mask) start first.
+    const int bh = blockIdx.x / p.num_cta_tiles;
+    const int ct = p.num_cta_tiles - 1 - static_cast<int>(blockIdx.x % p.num_cta_tiles);
+    const int m0 = ct * (QT * BM);
     const int n = p.n;
-    int jlo, jhi;
-    key_tile_range(m0, n, p.causal, p.window, jlo, jhi);
-    const int nt = jhi - jlo;  // >= 1: the diagonal tile always holds allowed keys
+    int jlo_s[QT], jhi_s[QT];
+#pragma unroll
+    for (int s = 0; s < QT; ++s) key_tile_range(m0 + s * BM, n, p.causal, p.window, jlo_s[s], jhi_s[s]);
+    // Union of the ranges: contiguous, starts with tile 0's, ends with the last
+    // non-empty tile's.
+    const int jlo = jlo_s[0];
+    const int jhi = (jhi_s[1] > jlo_s[1]) ? max(jhi_s[0], jhi_s[1]) : jhi_s[0];
+    const int nkv = jhi - jlo;  // key tiles loaded; >= 1
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(k_full(s), 1);
-            mbar_init(k_empty(s), 1);
-            mbar_init(v_full(s), 1);
-            mbar_init(v_empty(s), 1);
+        for (int s = 0; s < QT; ++s) {
+            mbar_init(q_full(s), 1);
+            mbar_init(s_full(s), 1);
+            mbar_init(p_full(s), BM);
+            mbar_init(o_done(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(s_full(b), 1);
-            mbar_init(p_full(b), BM);
+        for (int i = 0; i < NSLOT; ++i) {
+            mbar_init(kv_full(i), 1);
+            mbar_init(kv_empty(i), 1);
         }
-        mbar_init(o_done, 1);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 9 && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmO);
     }
-    if (warp == 5) {
+    if (warp == 8) {
         tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -208,76 +247,91 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const Waiter wt{abort_flag, p.status};
 
-    if (warp == 4) {
+    if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-            for (int b = 0; b < C::BOXES; ++b)
-                tma_load_3d(sQ + b * BOX_BYTES, &tmQ, q_full, b * BOX_COLS, m0, bh);
-            int kcount = 0, vcount = 0;
-            bool ok = true;
-            for (int t = 0; t < nt && ok; ++t) {
-                const int s = t % NS;
-                const uint32_t ph = (t / NS) & 1u;
-                const int k0 = (jlo + t) * BN;
-                if (t >= NS && !wt.wait(k_empty(s), ph ^ 1u)) { ok = false; break; }
-                mbar_arrive_expect_tx(k_full(s), C::TILE_BYTES);
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sK(s) + b * BOX_BYTES, &tmK, k_full(s), b * BOX_COLS, k0, bh);
-                ++kcount;
-                if (t >= NS && !wt.wait(v_empty(s), ph ^ 1u)) { ok = false; break; }
-                mbar_arrive_expect_tx(v_full(s), C::TILE_BYTES);
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sV(s) + b * BOX_BYTES, &tmV, v_full(s), b * BOX_COLS, k0, bh);
-                ++vcount;
-            }
-            if (!ok) {
-                // Let every copy issued into shared memory land before exiting.
-                wt.drain(q_full, 0);
-                for (int s = 0; s < NS; ++s) {
-                    if (kcount > s) wt.drain(k_full(s), (((kcount - 1 - s) / NS)) & 1u);
-                    if (vcount > s) wt.drain(v_full(s), (((vcount - 1 - s) / NS)) & 1u);
+            bool q_issued[QT];
+#pragma unroll
+            for (int s = 0; s < QT; ++s) {
+                q_issued[s] = jhi_s[s] > jlo_s[s];
+                if (q_issued[s]) {
+                    mbar_arrive_expect_tx(q_full(s), C::TILE_BYTES);
+                    for (int b = 0; b < C::BOXES; ++b)
+                        tma_load_3d(sQ(s) + b * BOX_BYTES, &tmQ, q_full(s), b * BOX_COLS, m0 + s * BM, bh);
                 }
             }
+            // item i: K of tile jlo + i/2 (i even) or V of it (i odd)
+            int issued = 0;
+            for (int i = 0; i < 2 * nkv; ++i) {
+                const int slot = i % NSLOT;
+                if (i >= NSLOT && !wt.wait(kv_empty(slot), ((i / NSLOT) & 1u) ^ 1u)) break;
+                mbar_arrive_expect_tx(kv_full(slot), C::TILE_BYTES);
+                const CUtensorMap *map = (i & 1) ? &tmV : &tmK;
+                const int k0 = (jlo + i / 2) * BN;
+                for (int b = 0; b < C::BOXES; ++b)
+                    tma_load_3d(sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
+                ++issued;
+            }
+            if (issued < 2 * nkv) {
+                // Aborted: let every copy issued into shared memory land first.
+#pragma unroll
+                for (int s = 0; s < QT; ++s)
+                    if (q_issued[s]) wt.drain(q_full(s), 0);
+                for (int slot = 0; slot < NSLOT; ++slot)
+                    if (issued > slot) wt.drain(kv_full(slot), (((issued - 1 - slot) / NSLOT)) & 1u);
+            }
         }
-    } else if (warp == 5) {
+    } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);   // P K-major, V MN-major
-            bool ok = wt.wait(q_full, 0);
+            bool ok = true;
+#pragma unroll
+            for (int s = 0; s < QT; ++s)
+                if (ok && jhi_s[s] > jlo_s[s]) ok = wt.wait(q_full(s), 0);
             tc_fence_after();
-            for (int t = 0; ok && t <= nt; ++t) {
-                if (t < nt) {
-                    const int s = t % NS;
-                    if (!wt.wait(k_full(s), (t / NS) & 1u)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t d_s = tmem + static_cast<uint32_t>(t & 1) * BN;
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t off = (k / 4) * BOX_BYTES + (k % 4) * 32;
-                        mma_bf16_ss(d_s, smem_desc_sw128(sQ + off, 16, 1024),
-                                    smem_desc_sw128(sK(s) + off, 16, 1024), idesc_qk, k > 0);
-                    }
-                    mma_commit(k_empty(s));
-                    mma_commit(s_full(t & 1));
+            for (int j = jlo; ok && j <= jhi; ++j) {
+                const int ik = 2 * (j - jlo);   // ring item of K_j
+                const int iv = ik - 1;          // ring item of V_{j-1}
+                if (j < jhi) {
+                    if (!wt.wait(kv_full(ik % NSLOT), (ik / NSLOT) & 1u)) { ok = false; break; }
                 }
-                if (t >= 1) {
-                    const int u = t - 1;
-                    const int s = u % NS;
-                    if (!wt.wait(p_full(u & 1), (u >> 1) & 1u)) { ok = false; break; }
-                    if (!wt.wait(v_full(s), (u / NS) & 1u)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a_p = tmem + static_cast<uint32_t>(u & 1) * BN;
-#pragma unroll
-                    for (int k = 0; k < BN / 16; ++k) {
-                        mma_bf16_ts(tmem + C::O_COL, a_p + k * 8,
-                                    smem_desc_sw128(sV(s) + k * 16 * 128, BOX_BYTES, 1024), idesc_pv,
-                                    (u > 0 || k > 0) ? 1u : 0u);
-                    }
-                    mma_commit(v_empty(s));
-                    mma_commit(o_done);
+                if (j > jlo) {
+                    if (!wt.wait(kv_full(iv % NSLOT), (iv / NSLOT) & 1u)) { ok = false; break; }
                 }
+                tc_fence_after();
+#pragma unroll
+                for (int s = 0; s < QT; ++s) {
+                    const uint32_t s_col = tmem + C::S_COL + s * BN;
+                    if (j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) {
+                        // O_s += P_s(j-1) V_{j-1}
+                        const int u = j - 1 - jlo_s[s];
+                        if (!wt.wait(p_full(s), u & 1u)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t vb = sKV(iv % NSLOT);
+#pragma unroll
+                        for (int k = 0; k < BN / 16; ++k)
+                            mma_bf16_ts(tmem + C::O_COL + s * D, s_col + k * 8,
+                                        smem_desc_sw128(vb + k * 16 * 128, BOX_BYTES, 1024), idesc_pv,
+                                        (u > 0 || k > 0) ? 1u : 0u);
+                        if (j == jhi_s[s]) mma_commit(o_done(s));
+                    }
+                    if (j >= jlo_s[s] && j < jhi_s[s]) {
+                        // S_s(j) = Q_s K_j^T
+                        const uint32_t kb = sKV(ik % NSLOT);
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t off = (k / 4) * BOX_BYTES + (k % 4) * 32;
+                            mma_bf16_ss(s_col, smem_desc_sw128(sQ(s) + off, 16, 1024),
+                                        smem_desc_sw128(kb + off, 16, 1024), idesc_qk, k > 0);
+                        }
+                        mma_commit(s_full(s));
+                    }
+                }
+                if (!ok) break;
+                if (j < jhi) mma_commit(kv_empty(ik % NSLOT));
+                if (j > jlo) mma_commit(kv_empty(iv % NSLOT));
             }
             // Every MMA this thread issued must finish before TMEM is freed.
             mma_commit(drain_bar);
@@ -285,130 +339,149 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ softmax
-        const int r = threadIdx.x;  // row in tile == TMEM lane
-        const int row = m0 + r;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int s = warp / 4;              // query tile of this warpgroup
+        const int r = threadIdx.x % BM;      // row in tile == TMEM lane
+        const int row = m0 + s * BM + r;
+        const int q0 = m0 + s * BM;          // first row of the tile
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+        const uint32_t s_base = lane_base + C::S_COL + s * BN;
+        const uint32_t o_base = lane_base + C::O_COL + s * D;
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
-        float mx = -CUDART_INF_F;  // running (possibly stale) max, log2 units
+        const int my_jlo = jlo_s[s], my_jhi = jhi_s[s];
+        float mx = -CUDART_INF_F;  // running max, log2 units
         float l = 0.f;             // running normaliser relative to mx
         bool ok = true;
 
-        for (int t = 0; t < nt; ++t) {
-            const int b = t & 1;
-            ok = __all_sync(0xffffffffu, wt.wait(s_full(b), (t >> 1) & 1u));
+        for (int j = my_jlo; j < my_jhi; ++j) {
+            const int u = j - my_jlo;
+            ok = __all_sync(0xffffffffu, wt.wait(s_full(s), u & 1u));
             if (!ok) break;
             tc_fence_after();
-            uint32_t s[BN];
+            uint32_t sv[BN];
 #pragma unroll
             for (int c = 0; c < BN; c += 32)
-                tmem_ld32(lane_base + b * BN + c, *reinterpret_cast<uint32_t(*)[32]>(&s[c]));
+                tmem_ld32(s_base + c, *reinterpret_cast<uint32_t(*)[32]>(&sv[c]));
 
-            const int k0 = (jlo + t) * BN;
-            const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > m0) ||
-                                   (window >= 0 && k0 < m0 + BM - 1 - window);
+            const int k0 = j * BN;
+            const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
+                                   (window >= 0 && k0 < q0 + BM - 1 - window);
             if (need_mask) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
                     const int key = k0 + c;
                     const bool allowed = key < n && (!causal || key <= row) &&
                                          (window < 0 || key >= row - window);
-                    if (!allowed) s[c] = f2u(-CUDART_INF_F);
+                    if (!allowed) sv[c] = f2u(-CUDART_INF_F);
                 }
             }
             float pm[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = u2f(s[i]);
+            for (int i = 0; i < 8; ++i) pm[i] = fmax3(u2f(sv[i]), u2f(sv[8 + i]), u2f(sv[16 + i]));
 #pragma unroll
-            for (int c = 8; c < BN; ++c) pm[c & 7] = fmaxf(pm[c & 7], u2f(s[c]));
-            const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            for (int c = 24; c < BN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], u2f(sv[c + i]), u2f(sv[c + 8 + i]));
+            const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
             const float mnew = tmax * sc;
             float alpha = 1.f;
-            bool rescale = false;
-            if (mnew > mx + RESCALE_THRESHOLD) {
+            const bool rescale = mnew > mx;
+            if (rescale) {
                 alpha = ex2_approx(mx - mnew);  // 0 when mx is -inf
                 mx = mnew;
-                rescale = true;
             }
             const float off = (mx == -CUDART_INF_F) ? 0.f : mx;  // no (-inf) - (-inf)
-            float ps[8];
+            const float2 sc2 = make_float2(sc, sc);
+            const float2 noff2 = make_float2(-off, -off);
+            float2 ps[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) ps[i] = 0.f;
+            for (int i = 0; i < 4; ++i) ps[i] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float e0 = ex2_approx(fmaf(u2f(s[c0 + 2 * i]), sc, -off));
-                    const float e1 = ex2_approx(fmaf(u2f(s[c0 + 2 * i + 1]), sc, -off));
-                    ps[(2 * i) & 7] += e0;
-                    ps[(2 * i + 1) & 7] += e1;
+                    const float2 x = ffma2(make_float2(u2f(sv[c0 + 2 * i]), u2f(sv[c0 + 2 * i + 1])), sc2, noff2);
+                    float e0, e1;
+                    if (C::EX2_EMU > 0 && !need_mask && (i % 8) < C::EX2_EMU) {
+                        ex2_poly_x2(x.x, x.y, e0, e1);
+                    } else {
+                        e0 = ex2_approx(x.x);
+                        e1 = ex2_approx(x.y);
+                    }
+                    ps[i & 3] = fadd2(ps[i & 3], make_float2(e0, e1));
                     pk[i] = pack_bf16x2(e0, e1);
                 }
-                tmem_st16(lane_base + b * BN + c0 / 2, pk);
+                tmem_st16(s_base + c0 / 2, pk);
             }
-            const float tsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-            l = l * alpha + tsum;
+            const float2 ps01 = fadd2(ps[0], ps[1]);
+            const float2 ps23 = fadd2(ps[2], ps[3]);
+            const float2 pst = fadd2(ps01, ps23);
+            l = fmaf(l, alpha, pst.x + pst.y);
 
-            if (t > 0) {
-                // O holds P_{t-1} V_{t-1} once that MMA is done; rescale if needed.
-                ok = __all_sync(0xffffffffu, wt.wait(o_done, (t - 1) & 1u));
-                if (!ok) break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
+            // O_s holds sum_{t<j} P_t V_t: PV_s(j-1) was issued before S_s(j)
+            // and has completed with it. Rescale when a row's max grew.
+            if (u > 0 && __any_sync(0xffffffffu, rescale)) {
+                const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
-                    for (int c = 0; c < D; c += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(lane_base + C::O_COL + c, o);
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_base + c, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = f2u(u2f(o[i]) * alpha);
-                        tmem_st32(lane_base + C::O_COL + c, o);
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 v = fmul2(make_float2(u2f(o[2 * i]), u2f(o[2 * i + 1])), a2);
+                        o[2 * i] = f2u(v.x);
+                        o[2 * i + 1] = f2u(v.y);
                     }
+                    tmem_st32(o_base + c, o);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(p_full(b));
+            mbar_arrive(p_full(s));
         }
-        if (ok) ok = __all_sync(0xffffffffu, wt.wait(o_done, (nt - 1) & 1u));
-        const bool all_ok = named_bar_and(1, BM, ok);
-        if (all_ok) {
-            tc_fence_after();
-            // Epilogue: O / l -> bf16 -> swizzled smem (the Q buffer, free now)
-            // -> TMA store; rows past n are clipped by the store.
-            const float inv_l = 1.f / l;
+        if (my_jhi > my_jlo) {
+            if (ok) ok = __all_sync(0xffffffffu, wt.wait(o_done(s), 0));
+            const bool all_ok = named_bar_and(1 + s, BM, ok);
+            if (all_ok) {
+                tc_fence_after();
+                // Epilogue: O / l -> bf16 -> swizzled smem (this tile's Q buffer,
+                // free once its last MMA is done) -> TMA store; rows past n are
+                // clipped by the store.
+                const float inv_l = 1.f / l;
+                const uint32_t stage = sQ(s);
 #pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + C::O_COL + c, o);
-                uint32_t pk[16];
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_base + c, o);
+                    uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l);
-                const uint32_t box = sQ + (c / BOX_COLS) * BOX_BYTES + r * 128;
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(u2f(o[2 * i]) * inv_l, u2f(o[2 * i + 1]) * inv_l);
+                    const uint32_t rowp = stage + (c / BOX_COLS) * BOX_BYTES + r * 128;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t chunk = ((c % BOX_COLS) / 8 + q) ^ (r & 7);
-                    st_shared_v4(box + chunk * 16, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t chunk = ((c % BOX_COLS) / 8 + q) ^ (r & 7);
+                        st_shared_v4(rowp + chunk * 16, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    }
                 }
+                fence_proxy_async_smem();
+                named_bar_sync(1 + s, BM);
+                if (r == 0) {
+                    for (int b = 0; b < C::BOXES; ++b)
+                        tma_store_3d(&tmO, stage + b * BOX_BYTES, b * BOX_COLS, q0, bh);
+                    tma_store_commit();
+                    tma_store_wait_read0();
+                }
+                if (row < n)
+                    p.lse[static_cast<size_t>(bh) * n + row] = (mx + __log2f(l)) * 0.69314718055994531f;
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, BM);
-            if (threadIdx.x == 0) {
-                for (int b = 0; b < C::BOXES; ++b)
-                    tma_store_3d(&tmO, sQ + b * BOX_BYTES, b * BOX_COLS, m0, bh);
-                tma_store_commit();
-                tma_store_wait_read0();
-            }
-            if (row < n)
-                p.lse[static_cast<size_t>(bh) * n + row] = (mx + __log2f(l)) * 0.69314718055994531f;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 8) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
