@@ -116,6 +116,14 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
         std::lock_guard<std::mutex> lk(g_mu);
         bool &set = g_smem_set[dev][D == 128 ? 1 : 0];
         if (!set) {
+            // The kernel moves registers between its warpgroups; that only
+            // works if it is launched with exactly the per-thread register
+            // count the split was computed for (else the raising warps wait
+            // forever). Refuse to launch a build that differs.
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D>) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
             if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Cfg::SMEM_BYTES) != cudaSuccess)

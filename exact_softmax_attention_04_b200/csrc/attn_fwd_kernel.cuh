@@ -11,7 +11,7 @@
 // online softmax trick"): the running output stays unnormalised and is
 // divided once, and only the current tile's scores ever live on chip.
 //
-// Roles (320 threads, 10 warps):
+// Roles (384 threads, 12 warps = 3 warpgroups, one warp of each per SMSP):
 //   warps 0-3  softmax for Q_0; warps 4-7 softmax for Q_1. Thread r of a
 //              warpgroup owns query row r (= TMEM lane r): it reads its S row,
 //              masks boundary tiles, updates (m, l), writes P (bf16) back into
@@ -20,6 +20,10 @@
 //   warp 8     MMA issuer (one elected lane) and TMEM owner.
 //   warp 9     TMA producer (one elected lane): Q_0, Q_1 once, then K_j, V_j
 //              alternately into a ring of NSLOT shared-memory slots.
+//   warps 10-11 idle (they complete the third warpgroup).
+// Registers: launched at 168 per thread; the softmax warpgroups raise theirs
+// to 232 (a 128-float S row plus its P stay in registers, no spills) and the
+// third warpgroup drops to 40: 2*128*232 + 128*40 = 384*168.
 // TMEM columns: S_0/P_0 [0,128), S_1/P_1 [128,256), O_0 [256, 256+D),
 // O_1 [256+D, 256+2D).
 // MMA issue order per key tile j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j). The
@@ -90,7 +94,12 @@ struct FwdCfg {
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL = 0;    // + s * BN
     static constexpr uint32_t O_COL = 256;  // + s * D
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
+    static constexpr uint32_t REGS_LAUNCH = 168;   // 65536 / 384, rounded down to 8
+    static constexpr uint32_t REGS_SOFTMAX = 232;
+    static constexpr uint32_t REGS_OTHER = 40;
+    static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER == THREADS * REGS_LAUNCH,
+                  "register split must use exactly the launch allocation");
     static constexpr int EX2_EMU = (D == 128) ? ATTN_EX2_EMU_D128 : ATTN_EX2_EMU_D64;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -197,7 +206,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
-    const int warp = threadIdx.x / 32;
+    // Warp index broadcast from lane 0, so the compiler knows it is uniform
+    // across the warp (role branches then keep warp-uniform values in
+    // uniform registers).
+    const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0);
     const int lane = threadIdx.x % 32;
 
     // Work: query-tile pairs of one head are adjacent in blockIdx (K/V reuse in
@@ -247,98 +259,115 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const Waiter wt{abort_flag, p.status};
 
-    if (warp == 9) {
+    if (warp >= 8) {
+      // Third warpgroup: TMA producer, MMA issuer and two idle warps.
+      regs_decrease<C::REGS_OTHER>();
+      const uint32_t leader = elect_one();
+      if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            bool q_issued[QT];
+        // The whole warp runs this loop (uniform operands); one lane issues.
+        bool q_issued[QT];
 #pragma unroll
-            for (int s = 0; s < QT; ++s) {
-                q_issued[s] = jhi_s[s] > jlo_s[s];
-                if (q_issued[s]) {
-                    mbar_arrive_expect_tx(q_full(s), C::TILE_BYTES);
-                    for (int b = 0; b < C::BOXES; ++b)
-                        tma_load_3d(sQ(s) + b * BOX_BYTES, &tmQ, q_full(s), b * BOX_COLS, m0 + s * BM, bh);
-                }
-            }
-            // item i: K of tile jlo + i/2 (i even) or V of it (i odd)
-            int issued = 0;
-            for (int i = 0; i < 2 * nkv; ++i) {
-                const int slot = i % NSLOT;
-                if (i >= NSLOT && !wt.wait(kv_empty(slot), ((i / NSLOT) & 1u) ^ 1u)) break;
-                mbar_arrive_expect_tx(kv_full(slot), C::TILE_BYTES);
-                const CUtensorMap *map = (i & 1) ? &tmV : &tmK;
-                const int k0 = (jlo + i / 2) * BN;
+        for (int s = 0; s < QT; ++s) {
+            q_issued[s] = jhi_s[s] > jlo_s[s];
+            if (q_issued[s]) {
+                mbar_arrive_expect_tx_if(leader, q_full(s), C::TILE_BYTES);
+#pragma unroll
                 for (int b = 0; b < C::BOXES; ++b)
-                    tma_load_3d(sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
-                ++issued;
-            }
-            if (issued < 2 * nkv) {
-                // Aborted: let every copy issued into shared memory land first.
-#pragma unroll
-                for (int s = 0; s < QT; ++s)
-                    if (q_issued[s]) wt.drain(q_full(s), 0);
-                for (int slot = 0; slot < NSLOT; ++slot)
-                    if (issued > slot) wt.drain(kv_full(slot), (((issued - 1 - slot) / NSLOT)) & 1u);
+                    tma_load_3d_if(leader, sQ(s) + b * BOX_BYTES, &tmQ, q_full(s), b * BOX_COLS,
+                                   m0 + s * BM, bh);
             }
         }
-    } else if (warp == 8) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);   // P K-major, V MN-major
-            bool ok = true;
+        // item i: K of tile jlo + i/2 (i even) or V of it (i odd)
+        int issued = 0;
+        for (int i = 0; i < 2 * nkv; ++i) {
+            const int slot = i % NSLOT;
+            if (i >= NSLOT &&
+                !__all_sync(0xffffffffu, wt.wait(kv_empty(slot), ((i / NSLOT) & 1u) ^ 1u)))
+                break;
+            mbar_arrive_expect_tx_if(leader, kv_full(slot), C::TILE_BYTES);
+            const CUtensorMap *map = (i & 1) ? &tmV : &tmK;
+            const int k0 = (jlo + i / 2) * BN;
+#pragma unroll
+            for (int b = 0; b < C::BOXES; ++b)
+                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
+            ++issued;
+        }
+        if (issued < 2 * nkv) {
+            // Aborted: let every copy issued into shared memory land first.
 #pragma unroll
             for (int s = 0; s < QT; ++s)
-                if (ok && jhi_s[s] > jlo_s[s]) ok = wt.wait(q_full(s), 0);
-            tc_fence_after();
-            for (int j = jlo; ok && j <= jhi; ++j) {
-                const int ik = 2 * (j - jlo);   // ring item of K_j
-                const int iv = ik - 1;          // ring item of V_{j-1}
-                if (j < jhi) {
-                    if (!wt.wait(kv_full(ik % NSLOT), (ik / NSLOT) & 1u)) { ok = false; break; }
-                }
-                if (j > jlo) {
-                    if (!wt.wait(kv_full(iv % NSLOT), (iv / NSLOT) & 1u)) { ok = false; break; }
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int s = 0; s < QT; ++s) {
-                    const uint32_t s_col = tmem + C::S_COL + s * BN;
-                    if (j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) {
-                        // O_s += P_s(j-1) V_{j-1}
-                        const int u = j - 1 - jlo_s[s];
-                        if (!wt.wait(p_full(s), u & 1u)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t vb = sKV(iv % NSLOT);
-#pragma unroll
-                        for (int k = 0; k < BN / 16; ++k)
-                            mma_bf16_ts(tmem + C::O_COL + s * D, s_col + k * 8,
-                                        smem_desc_sw128(vb + k * 16 * 128, BOX_BYTES, 1024), idesc_pv,
-                                        (u > 0 || k > 0) ? 1u : 0u);
-                        if (j == jhi_s[s]) mma_commit(o_done(s));
-                    }
-                    if (j >= jlo_s[s] && j < jhi_s[s]) {
-                        // S_s(j) = Q_s K_j^T
-                        const uint32_t kb = sKV(ik % NSLOT);
-#pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t off = (k / 4) * BOX_BYTES + (k % 4) * 32;
-                            mma_bf16_ss(s_col, smem_desc_sw128(sQ(s) + off, 16, 1024),
-                                        smem_desc_sw128(kb + off, 16, 1024), idesc_qk, k > 0);
-                        }
-                        mma_commit(s_full(s));
-                    }
-                }
-                if (!ok) break;
-                if (j < jhi) mma_commit(kv_empty(ik % NSLOT));
-                if (j > jlo) mma_commit(kv_empty(iv % NSLOT));
-            }
-            // Every MMA this thread issued must finish before TMEM is freed.
-            mma_commit(drain_bar);
-            wt.drain(drain_bar, 0);
+                if (q_issued[s]) wt.drain(q_full(s), 0);
+            for (int slot = 0; slot < NSLOT; ++slot)
+                if (issued > slot) wt.drain(kv_full(slot), (((issued - 1 - slot) / NSLOT)) & 1u);
         }
+      } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        // The whole warp runs this loop (uniform operands); one lane issues
+        // every MMA and commit, so the commits track all of its MMAs.
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);  // Q, K both K-major
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);   // P K-major, V MN-major
+        bool ok = true;
+#pragma unroll
+        for (int s = 0; s < QT; ++s)
+            if (ok && jhi_s[s] > jlo_s[s]) ok = __all_sync(0xffffffffu, wt.wait(q_full(s), 0));
+        tc_fence_after();
+        // Descriptors: the start-address field is addr >> 4 in the low 14
+        // bits, so adding (byte offset >> 4) moves a descriptor within
+        // shared memory (all addresses stay below 2^18).
+        const uint64_t kdesc0 = smem_desc_sw128(sKV(0), 16, 1024);
+        const uint64_t vdesc0 = smem_desc_sw128(sKV(0), BOX_BYTES, 1024);
+        for (int j = jlo; ok && j <= jhi; ++j) {
+            const int ik = 2 * (j - jlo);   // ring item of K_j
+            const int iv = ik - 1;          // ring item of V_{j-1}
+            if (j < jhi && !__all_sync(0xffffffffu, wt.wait(kv_full(ik % NSLOT), (ik / NSLOT) & 1u))) {
+                ok = false;
+                break;
+            }
+            if (j > jlo && !__all_sync(0xffffffffu, wt.wait(kv_full(iv % NSLOT), (iv / NSLOT) & 1u))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(((ik % NSLOT) * C::TILE_BYTES) >> 4);
+            const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(((iv % NSLOT) * C::TILE_BYTES) >> 4);
+#pragma unroll
+            for (int s = 0; s < QT; ++s) {
+                const uint32_t s_col = tmem + C::S_COL + s * BN;
+                if (j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) {
+                    // O_s += P_s(j-1) V_{j-1}: BN/16 MMAs of 16 keys each
+                    const int u = j - 1 - jlo_s[s];
+                    if (!__all_sync(0xffffffffu, wt.wait(p_full(s), u & 1u))) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t o_col = tmem + C::O_COL + s * D;
+#pragma unroll
+                    for (int k = 0; k < BN / 16; ++k)
+                        mma_bf16_ts_if(leader, o_col, s_col + k * 8, vdesc + static_cast<uint64_t>(k * 128),
+                                       idesc_pv, (u > 0 || k > 0) ? 1u : 0u);
+                    if (j == jhi_s[s]) mma_commit_if(leader, o_done(s));
+                }
+                if (j >= jlo_s[s] && j < jhi_s[s]) {
+                    // S_s(j) = Q_s K_j^T: D/16 MMAs of 16 columns each
+                    const uint64_t qdesc = smem_desc_sw128(sQ(s), 16, 1024);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                        mma_bf16_ss_if(leader, s_col, qdesc + off, kdesc + off, idesc_qk, k > 0 ? 1u : 0u);
+                    }
+                    mma_commit_if(leader, s_full(s));
+                }
+            }
+            if (!ok) break;
+            if (j < jhi) mma_commit_if(leader, kv_empty(ik % NSLOT));
+            if (j > jlo) mma_commit_if(leader, kv_empty(iv % NSLOT));
+        }
+        // Every MMA this warp issued must finish before TMEM is freed.
+        mma_commit_if(leader, drain_bar);
+        wt.drain(drain_bar, 0);
+      }
     } else {
         // ------------------------------------------------------------ softmax
+        regs_increase<C::REGS_SOFTMAX>();
         const int s = warp / 4;              // query tile of this warpgroup
         const int r = threadIdx.x % BM;      // row in tile == TMEM lane
         const int row = m0 + s * BM + r;
@@ -359,21 +388,19 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[BN];
-#pragma unroll
-            for (int c = 0; c < BN; c += 32)
-                tmem_ld32(s_base + c, *reinterpret_cast<uint32_t(*)[32]>(&sv[c]));
+            tmem_ld128(s_base, sv);
 
             const int k0 = j * BN;
             const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
                                    (window >= 0 && k0 < q0 + BM - 1 - window);
             if (need_mask) {
+                // Allowed keys of this row form one interval; in tile columns:
+                // [lo, hi] with key = k0 + column.
+                const int hi = min(causal ? row - k0 : BN - 1, n - 1 - k0);
+                const int lo = (window >= 0) ? row - window - k0 : 0;
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const int key = k0 + c;
-                    const bool allowed = key < n && (!causal || key <= row) &&
-                                         (window < 0 || key >= row - window);
-                    if (!allowed) sv[c] = f2u(-CUDART_INF_F);
-                }
+                for (int c = 0; c < BN; ++c)
+                    if (c > hi || c < lo) sv[c] = f2u(-CUDART_INF_F);
             }
             float pm[8];
 #pragma unroll
@@ -383,37 +410,34 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], u2f(sv[c + i]), u2f(sv[c + 8 + i]));
             const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-            const float mnew = tmax * sc;
-            float alpha = 1.f;
+            const float mnew = fmaxf(mx, tmax * sc);
             const bool rescale = mnew > mx;
-            if (rescale) {
-                alpha = ex2_approx(mx - mnew);  // 0 when mx is -inf
-                mx = mnew;
-            }
-            const float off = (mx == -CUDART_INF_F) ? 0.f : mx;  // no (-inf) - (-inf)
+            // alpha = 2^(m_old - m_new): 1 when the max did not grow, 0 when
+            // m_old = -inf; the selects avoid (-inf) - (-inf) and a branch.
+            const bool none_yet = (mnew == -CUDART_INF_F);
+            const float alpha = none_yet ? 1.f : ex2_approx(mx - mnew);
+            mx = mnew;
+            const float off = none_yet ? 0.f : mx;
             const float2 sc2 = make_float2(sc, sc);
             const float2 noff2 = make_float2(-off, -off);
             float2 ps[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) ps[i] = make_float2(0.f, 0.f);
+            uint32_t pk[BN / 2];
 #pragma unroll
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 x = ffma2(make_float2(u2f(sv[c0 + 2 * i]), u2f(sv[c0 + 2 * i + 1])), sc2, noff2);
-                    float e0, e1;
-                    if (C::EX2_EMU > 0 && !need_mask && (i % 8) < C::EX2_EMU) {
-                        ex2_poly_x2(x.x, x.y, e0, e1);
-                    } else {
-                        e0 = ex2_approx(x.x);
-                        e1 = ex2_approx(x.y);
-                    }
-                    ps[i & 3] = fadd2(ps[i & 3], make_float2(e0, e1));
-                    pk[i] = pack_bf16x2(e0, e1);
+            for (int i = 0; i < BN / 2; ++i) {
+                const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
+                float e0, e1;
+                if (C::EX2_EMU > 0 && !need_mask && (i % 8) < C::EX2_EMU) {
+                    ex2_poly_x2(x.x, x.y, e0, e1);
+                } else {
+                    e0 = ex2_approx(x.x);
+                    e1 = ex2_approx(x.y);
                 }
-                tmem_st16(s_base + c0 / 2, pk);
+                ps[i & 3] = fadd2(ps[i & 3], make_float2(e0, e1));
+                pk[i] = pack_bf16x2(e0, e1);
             }
+            tmem_st64(s_base, pk);
             const float2 ps01 = fadd2(ps[0], ps[1]);
             const float2 ps23 = fadd2(ps[2], ps[3]);
             const float2 pst = fadd2(ps01, ps23);
@@ -423,18 +447,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             // and has completed with it. Rescale when a row's max grew.
             if (u > 0 && __any_sync(0xffffffffu, rescale)) {
                 const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(o_base + c, o);
+                uint32_t o[D];
+                if constexpr (D == 128) tmem_ld128(o_base, o); else tmem_ld64(o_base, o);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 v = fmul2(make_float2(u2f(o[2 * i]), u2f(o[2 * i + 1])), a2);
-                        o[2 * i] = f2u(v.x);
-                        o[2 * i + 1] = f2u(v.y);
-                    }
-                    tmem_st32(o_base + c, o);
+                for (int i = 0; i < D / 2; ++i) {
+                    const float2 v = fmul2(make_float2(u2f(o[2 * i]), u2f(o[2 * i + 1])), a2);
+                    o[2 * i] = f2u(v.x);
+                    o[2 * i + 1] = f2u(v.y);
                 }
+                if constexpr (D == 128) tmem_st128(o_base, o); else tmem_st64(o_base, o);
             }
             tmem_wait_st();
             tc_fence_before();
