@@ -24,10 +24,11 @@ ATTN_ERR_INVALID = 1
 ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_CUDA = 3
 ATTN_ERR_TIMEOUT = 4
+ATTN_ERR_TOO_LARGE = 5
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_host_staging_release", "attn_sync_status",
-           "attn_strerror", "attn_attended_pairs")
+           "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc")
 
 
 class AttnError(RuntimeError):
@@ -48,6 +49,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd.restype = i
     lib.attn_fwd_host.argtypes = fwd_args
     lib.attn_fwd_host.restype = i
+    lib.attn_fwd_host_noalloc.argtypes = fwd_args
+    lib.attn_fwd_host_noalloc.restype = i
     lib.attn_host_staging_release.argtypes = []
     lib.attn_host_staging_release.restype = i
     lib.attn_sync_status.argtypes = [vp]

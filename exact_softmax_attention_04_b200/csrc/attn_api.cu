@@ -250,6 +250,7 @@ extern "C" const char *attn_strerror(int status)
     case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head size must be 64 or 128; a window needs causal=1)";
     case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
     case ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait; outputs are undefined";
+    case ATTN_ERR_TOO_LARGE: return "problem larger than the fixed scratch of attn_fwd_host_noalloc";
     default: return "unknown status";
     }
 }
@@ -261,4 +262,71 @@ extern "C" int64_t attn_attended_pairs(int64_t n, int causal, int64_t window)
         return (window + 1) * (window + 2) / 2 + (n - window - 1) * (window + 1);
     if (causal) return n * (n + 1) / 2;
     return n * n;
+}
+
+// ---------------------------------------------------------------------------
+// attn_fwd_host_noalloc: the host-buffer entry point without any allocation.
+// All of its device scratch sits in this file-scope array. In host code the
+// name g_noalloc_scratch is only a host-side stand-in, never a device address:
+// the address handed to copies and kernels comes from cudaGetSymbolAddress,
+// resolved once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void *g_noalloc_base[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on `dev` (the current device).
+int noalloc_base(int dev, char **out)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_base[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ATTN_ERR_CUDA;
+        g_noalloc_base[dev] = p;
+    }
+    *out = static_cast<char *>(g_noalloc_base[dev]);
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd_host_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                     int B, int H, int n, int d, float scale, int causal, int window,
+                                     void *stream)
+{
+    int rc = check_args(q, k, v, o, lse, B, H, n, d, scale, causal, window, false);
+    if (rc != ATTN_OK) return rc;
+    // Layout: [status word | q | k | v | o | lse], each part 256-byte aligned.
+    const size_t elems = static_cast<size_t>(B) * H * n * d;
+    const size_t tb = (elems * 2 + 255) & ~static_cast<size_t>(255);
+    const size_t lbytes = static_cast<size_t>(B) * H * n * 4;
+    const size_t lb = (lbytes + 255) & ~static_cast<size_t>(255);
+    if (elems > ATTN_NOALLOC_SCRATCH_BYTES || 256 + 4 * tb + lb > ATTN_NOALLOC_SCRATCH_BYTES)
+        return ATTN_ERR_TOO_LARGE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    char *base = nullptr;
+    rc = noalloc_base(dev, &base);
+    if (rc != ATTN_OK) return rc;
+    int *status = reinterpret_cast<int *>(base);
+    char *dq = base + 256, *dk = dq + tb, *dv = dk + tb, *dout = dv + tb;
+    float *dl = reinterpret_cast<float *>(dout + tb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // The status word keeps the previous call's value: clear it first.
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess ||
+        cudaMemcpyAsync(dq, q, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    rc = (d == 64) ? launch_fwd<64>(dq, dk, dv, dout, dl, B, H, n, scale, causal, window, st, dev, status)
+                   : launch_fwd<128>(dq, dk, dv, dout, dl, B, H, n, scale, causal, window, st, dev, status);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o, dout, elems * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(lse, dl, lbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+    return h != 0 ? ATTN_ERR_TIMEOUT : ATTN_OK;
 }

@@ -65,7 +65,8 @@ typedef enum {
     ATTN_ERR_INVALID = 1,     /* a bad argument; nothing was enqueued           */
     ATTN_ERR_UNSUPPORTED = 2, /* valid but not provided (d not 64/128, ...)     */
     ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed              */
-    ATTN_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (device side)  */
+    ATTN_ERR_TIMEOUT = 4,     /* a kernel's bounded wait expired (device side)  */
+    ATTN_ERR_TOO_LARGE = 5    /* exceeds the fixed scratch of attn_fwd_host_noalloc */
 } attn_status;
 
 /*
@@ -108,6 +109,39 @@ ATTN_API int attn_fwd_host(const void *q, const void *k, const void *v, void *o,
 
 /* Frees this device's attn_fwd_host staging buffers (synchronizes the device). */
 ATTN_API int attn_host_staging_release(void);
+
+/* Size of the fixed device scratch of attn_fwd_host_noalloc, per device. */
+#define ATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * attn_fwd_host_noalloc - attn_fwd_host for callers that must not allocate
+ * device memory. The pages have no counterpart to it: it exists for programs
+ * that run under a fixed device-memory budget owned by someone else, or that
+ * cannot afford the device-wide synchronisation cudaMalloc/cudaFree may
+ * cause, and therefore cannot let a library allocate on their behalf.
+ *
+ * Same arguments and result as attn_fwd_host (host buffers in, host buffers
+ * out), but every device-side scratch byte it uses (the staging copies of q,
+ * k, v, o, lse and the kernel's status word) lives in one statically sized
+ * device array of ATTN_NOALLOC_SCRATCH_BYTES that the library holds on every
+ * device that loads it, until the process exits. It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *
+ *   Limit: 4 * B*H*n*d*2 + B*H*n*4 bytes (each part rounded up to 256) plus
+ *          256 must fit in ATTN_NOALLOC_SCRATCH_BYTES; larger problems return
+ *          ATTN_ERR_TOO_LARGE before any device work.
+ *   Synchronous: returns once o and lse are written (it synchronizes
+ *          `stream`), with ATTN_ERR_TIMEOUT if the kernel gave up a wait.
+ *   Set-up: the first call on a device looks up the array's device address
+ *          (cudaGetSymbolAddress) with that device current; make that first
+ *          call before any stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps the last
+ *          call's contents; calls whose work overlaps on the GPU (other
+ *          streams or threads) race and must be serialised by the caller.
+ */
+ATTN_API int attn_fwd_host_noalloc(const void *q, const void *k, const void *v, void *o,
+                                   float *lse, int B, int H, int n, int d, float scale,
+                                   int causal, int window, void *stream);
 
 /*
  * attn_sync_status - synchronize `stream`, then read and clear this device's
