@@ -38,6 +38,7 @@
 // for its own copies and MMAs in flight, frees TMEM and returns.
 #pragma once
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <math_constants.h>
 
 #include "sm100.cuh"
@@ -61,10 +62,10 @@ constexpr int STATUS_WAIT_TIMEOUT = 1;
 // Exponentials computed on the FMA pipe instead of the MUFU unit: out of every
 // 8 pairs of a row chunk, the first ATTN_EX2_EMU pairs use the polynomial.
 #ifndef ATTN_EX2_EMU_D64
-#define ATTN_EX2_EMU_D64 0
+#define ATTN_EX2_EMU_D64 2
 #endif
 #ifndef ATTN_EX2_EMU_D128
-#define ATTN_EX2_EMU_D128 0
+#define ATTN_EX2_EMU_D128 2
 #endif
 
 struct FwdParams {
@@ -87,13 +88,22 @@ struct FwdCfg {
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = Q_OFF + QT * TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
-    // q_full[QT], kv_full[NSLOT], kv_empty[NSLOT], s_full[QT], p_full[QT], o_done[QT], drain
-    static constexpr int NUM_BARS = QT + 2 * NSLOT + 3 * QT + 1;
+    // q_full[QT], kv_full[NSLOT], kv_empty[NSLOT], s_full[QT], p_full[QT], o_done[QT],
+    // s_free[QT], pv_done[QT], drain
+    static constexpr int NUM_BARS = QT + 2 * NSLOT + 5 * QT + 1;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + 1 KB alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t S_COL = 0;    // + s * BN
     static constexpr uint32_t O_COL = 256;  // + s * D
+    // With D = 64 TMEM has room for P buffers of their own (64 columns of
+    // packed bf16 per tile), so S(j+1) can be computed as soon as the softmax
+    // has read S(j): the MMA round trip leaves the softmax's critical path.
+    // With D = 128 TMEM is full and P overwrites its S.
+    static constexpr bool SPLIT_P = (D == 64);
+    static constexpr uint32_t P_COL = SPLIT_P ? 256 + QT * D : S_COL;  // + s * (SPLIT_P ? BN/2 : BN)
+    static constexpr uint32_t P_STRIDE = SPLIT_P ? BN / 2 : BN;
+    static_assert(!SPLIT_P || P_COL + QT * P_STRIDE <= TMEM_COLS, "TMEM budget");
     static constexpr int THREADS = 384;
     static constexpr uint32_t REGS_LAUNCH = 168;   // 65536 / 384, rounded down to 8
     static constexpr uint32_t REGS_SOFTMAX = 232;
@@ -202,7 +212,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     auto s_full = [&](int s) { return bars + 8u * (QT + 2 * NSLOT + s); };
     auto p_full = [&](int s) { return bars + 8u * (2 * QT + 2 * NSLOT + s); };
     auto o_done = [&](int s) { return bars + 8u * (3 * QT + 2 * NSLOT + s); };
-    const uint32_t drain_bar = bars + 8u * (4 * QT + 2 * NSLOT);
+    auto s_free = [&](int s) { return bars + 8u * (4 * QT + 2 * NSLOT + s); };
+    auto pv_done = [&](int s) { return bars + 8u * (5 * QT + 2 * NSLOT + s); };
+    const uint32_t drain_bar = bars + 8u * (6 * QT + 2 * NSLOT);
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
@@ -234,6 +246,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             mbar_init(s_full(s), 1);
             mbar_init(p_full(s), BM);
             mbar_init(o_done(s), 1);
+            mbar_init(s_free(s), BM);
+            mbar_init(pv_done(s), 1);
         }
         for (int i = 0; i < NSLOT; ++i) {
             mbar_init(kv_full(i), 1);
@@ -331,30 +345,55 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             tc_fence_after();
             const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(((ik % NSLOT) * C::TILE_BYTES) >> 4);
             const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(((iv % NSLOT) * C::TILE_BYTES) >> 4);
+            // O_s += P_s(j-1) V_{j-1}: BN/16 MMAs of 16 keys each
+            auto issue_pv = [&](int s) -> bool {
+                const int u = j - 1 - jlo_s[s];
+                if (!__all_sync(0xffffffffu, wt.wait(p_full(s), u & 1u))) return false;
+                tc_fence_after();
+                const uint32_t o_col = tmem + C::O_COL + s * D;
+                const uint32_t p_col = tmem + C::P_COL + s * C::P_STRIDE;
 #pragma unroll
-            for (int s = 0; s < QT; ++s) {
-                const uint32_t s_col = tmem + C::S_COL + s * BN;
-                if (j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) {
-                    // O_s += P_s(j-1) V_{j-1}: BN/16 MMAs of 16 keys each
+                for (int k = 0; k < BN / 16; ++k)
+                    mma_bf16_ts_if(leader, o_col, p_col + k * 8, vdesc + static_cast<uint64_t>(k * 128),
+                                   idesc_pv, (u > 0 || k > 0) ? 1u : 0u);
+                if constexpr (C::SPLIT_P) mma_commit_if(leader, pv_done(s));
+                if (j == jhi_s[s]) mma_commit_if(leader, o_done(s));
+                return true;
+            };
+            // S_s(j) = Q_s K_j^T: D/16 MMAs of 16 columns each
+            auto issue_s = [&](int s) -> bool {
+                if constexpr (C::SPLIT_P) {
+                    // the softmax must have read S_s(j-1) out of TMEM
                     const int u = j - 1 - jlo_s[s];
-                    if (!__all_sync(0xffffffffu, wt.wait(p_full(s), u & 1u))) { ok = false; break; }
+                    if (u >= 0 && !__all_sync(0xffffffffu, wt.wait(s_free(s), u & 1u))) return false;
                     tc_fence_after();
-                    const uint32_t o_col = tmem + C::O_COL + s * D;
-#pragma unroll
-                    for (int k = 0; k < BN / 16; ++k)
-                        mma_bf16_ts_if(leader, o_col, s_col + k * 8, vdesc + static_cast<uint64_t>(k * 128),
-                                       idesc_pv, (u > 0 || k > 0) ? 1u : 0u);
-                    if (j == jhi_s[s]) mma_commit_if(leader, o_done(s));
                 }
-                if (j >= jlo_s[s] && j < jhi_s[s]) {
-                    // S_s(j) = Q_s K_j^T: D/16 MMAs of 16 columns each
-                    const uint64_t qdesc = smem_desc_sw128(sQ(s), 16, 1024);
+                const uint32_t s_col = tmem + C::S_COL + s * BN;
+                const uint64_t qdesc = smem_desc_sw128(sQ(s), 16, 1024);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
-                        mma_bf16_ss_if(leader, s_col, qdesc + off, kdesc + off, idesc_qk, k > 0 ? 1u : 0u);
-                    }
-                    mma_commit_if(leader, s_full(s));
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                    mma_bf16_ss_if(leader, s_col, qdesc + off, kdesc + off, idesc_qk, k > 0 ? 1u : 0u);
+                }
+                mma_commit_if(leader, s_full(s));
+                return true;
+            };
+            if constexpr (C::SPLIT_P) {
+                // S_0(j), S_1(j), then PV_0(j-1), PV_1(j-1): S(j) goes out as soon as
+                // S(j-1) has been read, long before P(j-1) is ready.
+#pragma unroll
+                for (int s = 0; s < QT; ++s)
+                    if (ok && j >= jlo_s[s] && j < jhi_s[s]) ok = issue_s(s);
+#pragma unroll
+                for (int s = 0; s < QT; ++s)
+                    if (ok && j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) ok = issue_pv(s);
+            } else {
+                // PV_0(j-1), S_0(j), PV_1(j-1), S_1(j): S_s(j) overwrites P_s(j-1) in
+                // TMEM, so it must follow PV_s(j-1) (MMAs complete in issue order).
+#pragma unroll
+                for (int s = 0; s < QT; ++s) {
+                    if (ok && j - 1 >= jlo_s[s] && j - 1 < jhi_s[s]) ok = issue_pv(s);
+                    if (ok && j >= jlo_s[s] && j < jhi_s[s]) ok = issue_s(s);
                 }
             }
             if (!ok) break;
@@ -375,6 +414,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
         const uint32_t s_base = lane_base + C::S_COL + s * BN;
         const uint32_t o_base = lane_base + C::O_COL + s * D;
+        const uint32_t p_base = lane_base + C::P_COL + s * C::P_STRIDE;
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
         const int my_jlo = jlo_s[s], my_jhi = jhi_s[s];
@@ -389,6 +429,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             tc_fence_after();
             uint32_t sv[BN];
             tmem_ld128(s_base, sv);
+            if constexpr (C::SPLIT_P) {
+                // S_s is in registers: the MMA warp may overwrite it with S_s(j+1).
+                tc_fence_before();
+                mbar_arrive(s_free(s));
+            }
 
             const int k0 = j * BN;
             const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
@@ -404,12 +449,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             }
             float pm[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = fmax3(u2f(sv[i]), u2f(sv[8 + i]), u2f(sv[16 + i]));
+            for (int i = 0; i < 8; ++i) pm[i] = fmaxf(u2f(sv[i]), u2f(sv[8 + i]));
 #pragma unroll
-            for (int c = 24; c < BN; c += 16)
+            for (int c = 16; c < BN; c += 8)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], u2f(sv[c + i]), u2f(sv[c + 8 + i]));
-            const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+                for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], u2f(sv[c + i]));
+            const float tmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             const float mnew = fmaxf(mx, tmax * sc);
             const bool rescale = mnew > mx;
             // alpha = 2^(m_old - m_new): 1 when the max did not grow, 0 when
@@ -424,27 +470,52 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) ps[i] = make_float2(0.f, 0.f);
             uint32_t pk[BN / 2];
+            // One straight-line body per case (no branch inside the unrolled
+            // loop, so MUFU and FMA work can be interleaved freely). Masked
+            // tiles always use the MUFU: the polynomial clamps at 2^-125.
+            auto exps = [&](auto emu) {
+                constexpr int EMU = decltype(emu)::value;
 #pragma unroll
-            for (int i = 0; i < BN / 2; ++i) {
-                const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
-                float e0, e1;
-                if (C::EX2_EMU > 0 && !need_mask && (i % 8) < C::EX2_EMU) {
-                    ex2_poly_x2(x.x, x.y, e0, e1);
-                } else {
-                    e0 = ex2_approx(x.x);
-                    e1 = ex2_approx(x.y);
+                for (int i = 0; i < BN / 2; ++i) {
+                    const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
+                    float e0, e1;
+                    if constexpr (EMU > 0) {
+                        if ((i % 8) < EMU) {
+                            ex2_poly_x2(x.x, x.y, e0, e1);
+                        } else {
+                            e0 = ex2_approx(x.x);
+                            e1 = ex2_approx(x.y);
+                        }
+                    } else {
+                        e0 = ex2_approx(x.x);
+                        e1 = ex2_approx(x.y);
+                    }
+                    ps[i & 3] = fadd2(ps[i & 3], make_float2(e0, e1));
+                    pk[i] = pack_bf16x2(e0, e1);
                 }
-                ps[i & 3] = fadd2(ps[i & 3], make_float2(e0, e1));
-                pk[i] = pack_bf16x2(e0, e1);
+            };
+            if (C::EX2_EMU == 0 || need_mask)
+                exps(std::integral_constant<int, 0>{});
+            else
+                exps(std::integral_constant<int, C::EX2_EMU>{});
+            if constexpr (C::SPLIT_P) {
+                // P_s(j) reuses P_s(j-1)'s columns and O_s is about to be
+                // rescaled: PV_s(j-1) must be complete.
+                if (u > 0) {
+                    ok = __all_sync(0xffffffffu, wt.wait(pv_done(s), (u - 1) & 1u));
+                    if (!ok) break;
+                    tc_fence_after();
+                }
             }
-            tmem_st64(s_base, pk);
+            tmem_st64(p_base, pk);
             const float2 ps01 = fadd2(ps[0], ps[1]);
             const float2 ps23 = fadd2(ps[2], ps[3]);
             const float2 pst = fadd2(ps01, ps23);
             l = fmaf(l, alpha, pst.x + pst.y);
 
-            // O_s holds sum_{t<j} P_t V_t: PV_s(j-1) was issued before S_s(j)
-            // and has completed with it. Rescale when a row's max grew.
+            // O_s holds sum_{t<j} P_t V_t: PV_s(j-1) has completed (waited for
+            // above with separate P buffers; otherwise it was issued before
+            // S_s(j) and completed with it). Rescale when a row's max grew.
             if (u > 0 && __any_sync(0xffffffffu, rescale)) {
                 const float2 a2 = make_float2(alpha, alpha);
                 uint32_t o[D];
