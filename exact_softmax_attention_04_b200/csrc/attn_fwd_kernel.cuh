@@ -60,12 +60,12 @@ constexpr int STATUS_WAIT_TIMEOUT = 1;
 // dominant term: too much for peaked rows.)
 
 // Exponentials computed on the FMA pipe instead of the MUFU unit: out of every
-// 8 pairs of a row chunk, the first ATTN_EX2_EMU pairs use the polynomial.
+// 16 pairs of a row, the first ATTN_EX2_EMU_D* pairs use the polynomial.
 #ifndef ATTN_EX2_EMU_D64
-#define ATTN_EX2_EMU_D64 2
+#define ATTN_EX2_EMU_D64 3
 #endif
 #ifndef ATTN_EX2_EMU_D128
-#define ATTN_EX2_EMU_D128 2
+#define ATTN_EX2_EMU_D128 4
 #endif
 
 struct FwdParams {
@@ -179,8 +179,8 @@ __device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float &y0, float
     x0 = fmaxf(x0, -125.0f);
     x1 = fmaxf(x1, -125.0f);
     const float2 t = fadd2(make_float2(x0, x1), make_float2(kRound, kRound));
-    const float2 r = fadd2(t, make_float2(-kRound, -kRound));        // round(x)
-    const float2 f = fadd2(make_float2(x0, x1), make_float2(-r.x, -r.y));
+    const float2 r = fsub2(t, make_float2(kRound, kRound));          // round(x)
+    const float2 f = fsub2(make_float2(x0, x1), r);
     float2 p = ffma2(make_float2(0.05517167f, 0.05517167f), f, make_float2(0.24261113f, 0.24261113f));
     p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
     p = ffma2(p, f, make_float2(0.99992806f, 0.99992806f));
@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
                     float e0, e1;
                     if constexpr (EMU > 0) {
-                        if ((i % 8) < EMU) {
+                        if ((i % 16) < EMU) {
                             ex2_poly_x2(x.x, x.y, e0, e1);
                         } else {
                             e0 = ex2_approx(x.x);
