@@ -372,6 +372,50 @@ def run_ours(args, wl, world, rank, local):
     return 0
 
 
+def run_sweep(args):
+    """Kernel time of every target workload (one line each): TFLOP/s on
+    unmasked FLOPs, % of the measured peak and HBM GB/s on the minimum bytes
+    (Q, K, V read once, O and LSE written once). Informational table; the
+    parity of each of these workloads is checked by the test suite."""
+    import exact_softmax_attention_04_b200 as attn
+    from exact_softmax_attention_04_b200 import synth
+    torch.cuda.set_device(0)
+    bf16_peak, hbm_peak, peak_src = peaks()
+    wls = [synth.SMALL_CAUSAL, synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072] + synth.sweep()
+    for wl in wls:
+        q, k, v = synth.make_inputs(wl)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        o = torch.empty_like(qd)
+        lse = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, device="cuda")
+        flops = synth.unmasked_flops(wl)
+        min_bytes = 4 * q.numel() * 2 + lse.numel() * 4
+        # L2 flush buffer (256 MB) between timed launches for small problems
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        f = lambda: attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        for _ in range(args.warmup):
+            f()
+        st = attn.sync_status()
+        times = []
+        for _ in range(max(3, args.steps)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            f()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        tf = flops / (ms / 1e3) / 1e12
+        print(json.dumps({"workload": wl.name, "ms": ms, "tflops": tf,
+                          "pct_of_peak": 100 * tf / bf16_peak, "hbm_gbs": min_bytes / (ms / 1e3) / 1e9,
+                          "pct_of_hbm": 100 * min_bytes / (ms / 1e3) / 1e9 / hbm_peak,
+                          "status": st, "l2": "flushed (256 MB write) before each timed launch",
+                          "peak_source": peak_src}), flush=True)
+        del qd, kd, vd, o, lse, flush
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,12 +425,16 @@ def main():
     ap.add_argument("--workload", default="B8-H8-n8192-d64-none")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every target workload (kernel only, median of --steps, L2 flushed)")
     ap.add_argument("--profile", action="store_true",
                     help="timed kernel launches only (no e2e, CPU baseline or clock sampling): "
                          "the command profiled under ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        return run_sweep(args)
     from exact_softmax_attention_04_b200 import synth
     wl = synth.by_name(args.workload)
     if wl is None:

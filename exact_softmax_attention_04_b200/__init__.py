@@ -38,11 +38,16 @@ class AttnError(RuntimeError):
 
 
 def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+    return load_library(LIB_PATH)
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """ctypes handle of a libattn_b200 build at ``path`` with argument types set."""
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m exact_softmax_attention_04_b200.build_lib` "
+            f"{path} is missing: build it with `python -m exact_softmax_attention_04_b200.build_lib` "
             "(there is no CPU fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, i, f, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64
     fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.attn_fwd.argtypes = fwd_args

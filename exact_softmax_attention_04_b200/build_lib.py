@@ -52,6 +52,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_variant(out_path: str, defines) -> str:
+    """Build the same sources with extra preprocessor definitions into
+    ``out_path`` (used by the fault-injection test; never the library)."""
+    cmd = [_nvcc()] + NVCC_FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
+    cmd += [f"-D{d}" for d in defines]
+    cmd += ["-o", str(out_path)] + SOURCES
+    subprocess.check_call(cmd)
+    return str(out_path)
+
+
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")

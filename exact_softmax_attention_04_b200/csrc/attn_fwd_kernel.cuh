@@ -296,6 +296,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         int issued = 0;
         for (int i = 0; i < 2 * nkv; ++i) {
             const int slot = i % NSLOT;
+#ifdef ATTN_FAULT_DROP_FIRST_V
+            // Test hook (never defined in the library build): the V tile of
+            // the first key tile is never loaded, so the MMA warp's wait on it
+            // must expire and the kernel must stop cleanly.
+            if (i == 1) {
+                ++issued;
+                continue;
+            }
+#endif
             if (i >= NSLOT &&
                 !__all_sync(0xffffffffu, wt.wait(kv_empty(slot), ((i / NSLOT) & 1u) ^ 1u)))
                 break;

@@ -1,0 +1,49 @@
+"""Failure detection without faulting the GPU.
+
+Every wait in the kernel is bounded (about one second). A build with the
+test-only ATTN_FAULT_DROP_FIRST_V hook never loads the first V tile, so the
+MMA warp's wait for it must expire: the kernel then sets the device status
+word, stops all roles, waits (bounded) for what it issued, frees TMEM and
+returns. The host must read ATTN_ERR_TIMEOUT, the status must clear, and the
+CUDA context must stay usable for a correct computation afterwards.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+from exact_softmax_attention_04_b200 import synth
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def test_expired_wait_reports_timeout_and_context_survives(tmp_path, oracle_mod):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import exact_softmax_attention_04_b200 as pkg
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    fault_lib = pkg.load_library(build_lib.build_variant(tmp_path / "libattn_fault.so",
+                                                         ["ATTN_FAULT_DROP_FIRST_V"]))
+    # one CTA (n = 256: two 128-row tiles), several key tiles
+    q, k, v = synth.make_qkv(1, 1, 256, 64, seed=50)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((1, 1, 256), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.time()
+    rc = fault_lib.attn_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            1, 1, 256, 64, 0.125, 0, -1, stream)
+    assert rc == pkg.ATTN_OK
+    st = fault_lib.attn_sync_status(stream)
+    elapsed = time.time() - t0
+    assert st == pkg.ATTN_ERR_TIMEOUT, pkg.strerror(st)
+    assert elapsed < 30.0
+    assert fault_lib.attn_sync_status(stream) == pkg.ATTN_OK  # read-and-clear
+    # the context is intact: the normal library computes the same problem correctly
+    o2, lse2 = pkg.attn_fwd(qd, kd, vd, 0.125, False, -1)
+    assert pkg.sync_status() == pkg.ATTN_OK
+    o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, 0.125, False, -1)
+    assert_close(o2.float().cpu().numpy(), lse2.cpu().numpy(), o_ref, lse_ref, "after timeout")
