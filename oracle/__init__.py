@@ -45,6 +45,9 @@ def _load():
         lib.oracle_attn_rows_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, ip,
                                              vp, i64, vp, vp, vp]
         lib.oracle_attn_rows_f64.restype = ip
+        lib.oracle_attn_rows_gqa_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, dbl, ip, i64,
+                                                 ip, vp, i64, vp, vp, vp]
+        lib.oracle_attn_rows_gqa_f64.restype = ip
         lib.oracle_attn_fwd_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, vp, vp]
         lib.oracle_attn_fwd_f64.restype = ip
         lib.oracle_matmul_f64.argtypes = [i64, i64, i64, vp, ip, vp, ip, vp]
@@ -83,6 +86,27 @@ def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
     if rc != 0:
         raise ValueError(f"oracle_attn_rows_f64 rejected its arguments (rc={rc})")
     return o, lse, w
+
+
+def attn_rows_gqa(q, k, v, scale: float, causal: bool, window: int, rows,
+                  kernel: int = KERNEL_SOFTMAX) -> Tuple[np.ndarray, np.ndarray]:
+    """Grouped-query form: q [B, H, n, d], k and v [B, Hkv, n, d], Hkv | H.
+    O (nrows x d) and LSE (nrows) for flat query rows (b*H + h)*n + i."""
+    lib = _load()
+    B, H, n, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k and v must be [B, Hkv, n, d]")
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.empty((rows.size, d), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    rc = lib.oracle_attn_rows_gqa_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, Hkv, n, d,
+                                      float(scale), int(bool(causal)), int(window), int(kernel),
+                                      rows.ctypes.data, rows.size, o.ctypes.data, lse.ctypes.data, None)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_rows_gqa_f64 rejected its arguments (rc={rc})")
+    return o, lse
 
 
 def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1

@@ -31,6 +31,11 @@
  * There is no tiling, no online rescaling and no reordering beyond the
  * definition. OpenMP spreads independent rows over host cores.
  *
+ * Grouped-query attention ("week17 efficiency attention", MQA / GQA
+ * section): K and V have H_kv heads, H_kv divides H, and query head h reads
+ * key/value head h / (H / H_kv); H_kv = 1 is multi-query attention and
+ * H_kv = H is ordinary multi-head attention.
+ *
  * The "identity" kernel (ORACLE_KERNEL_IDENTITY) replaces the softmax weight
  * exp(s_ij - M_i)/Z_i by the raw score s_ij and uses no mask: it yields the
  * unnormalised product (Q K^T) V * scale, which the associativity identity
@@ -106,8 +111,9 @@ int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned c
 }
 
 /*
- * Attention for a list of rows.
- *   q, k, v : bf16 bit patterns, contiguous [B, H, n, d]
+ * Attention for a list of rows, grouped-query form.
+ *   q       : bf16 bit patterns, contiguous [B, H, n, d]
+ *   k, v    : bf16 bit patterns, contiguous [B, Hkv, n, d]; Hkv divides H
  *   rows    : flat row ids r = (b*H + h)*n + i, nrows of them
  *   o       : nrows x d   fp64 output (row-major, in the order of rows)
  *   lse     : nrows       fp64 output (may be NULL)
@@ -115,13 +121,15 @@ int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned c
  *   kernel  : ORACLE_KERNEL_SOFTMAX or ORACLE_KERNEL_IDENTITY
  * window >= 0 requires causal. Returns 0 on success, nonzero on bad input.
  */
-int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                         int64_t B, int64_t H, int64_t n, int64_t d, double scale,
-                         int causal, int64_t window, int kernel,
-                         const int64_t *rows, int64_t nrows,
-                         double *o, double *lse, double *weights)
+int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             int64_t B, int64_t H, int64_t Hkv, int64_t n, int64_t d,
+                             double scale, int causal, int64_t window, int kernel,
+                             const int64_t *rows, int64_t nrows,
+                             double *o, double *lse, double *weights)
 {
     if (!q || !k || !v || !o || (!rows && nrows) || B <= 0 || H <= 0 || n <= 0 || d <= 0)
+        return 1;
+    if (Hkv <= 0 || H % Hkv != 0)
         return 1;
     if (window >= 0 && !causal)
         return 1;
@@ -147,8 +155,10 @@ int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v
             for (int64_t r = 0; r < nrows; ++r) {
                 int64_t bh = rows[r] / n;
                 int64_t i = rows[r] % n;
-                const uint16_t *Kh = k + bh * n * d;
-                const uint16_t *Vh = v + bh * n * d;
+                /* key/value head of query head h = bh % H in batch b = bh / H */
+                int64_t bkv = (bh / H) * Hkv + (bh % H) / (H / Hkv);
+                const uint16_t *Kh = k + bkv * n * d;
+                const uint16_t *Vh = v + bkv * n * d;
                 for (int64_t c = 0; c < d; ++c)
                     qi[c] = bf16_to_f64(q[(bh * n + i) * d + c]);
 
@@ -212,6 +222,17 @@ int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v
         free(allowed);
     }
     return bad ? 2 : 0;
+}
+
+/* Multi-head attention (Hkv = H) for a list of rows; arguments as above. */
+int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         int64_t B, int64_t H, int64_t n, int64_t d, double scale,
+                         int causal, int64_t window, int kernel,
+                         const int64_t *rows, int64_t nrows,
+                         double *o, double *lse, double *weights)
+{
+    return oracle_attn_rows_gqa_f64(q, k, v, B, H, H, n, d, scale, causal, window, kernel,
+                                    rows, nrows, o, lse, weights);
 }
 
 /* Every row of every head: o is [B, H, n, d] fp64, lse is [B, H, n] fp64. */

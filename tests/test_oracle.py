@@ -278,3 +278,51 @@ def test_pair_count_matches_explicit_masks(oracle_mod):
         for causal, window in [(False, -1), (True, -1), (True, 0), (True, 3), (True, 128), (True, 500)]:
             cnt = sum(int(oracle_mod.mask_row(n, i, causal, window).sum()) for i in range(n))
             assert cnt == synth.attended_pairs_per_head(n, causal, window)
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+def _brute_gqa(q, k, v, scale, causal, window):
+    """Textbook GQA: query head h uses key/value head h // (H // Hkv)."""
+    H, Hkv = q.shape[1], k.shape[1]
+    idx = torch.arange(H) // (H // Hkv)
+    return _brute(q, k[:, idx], v[:, idx], scale, causal, window)
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (6, 3), (4, 1)])
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 5)])
+def test_gqa_oracle_matches_brute_force(oracle_mod, H, Hkv, causal, window):
+    n, d = 37, 16
+    q, _, _ = synth.make_qkv(2, H, n, d, seed=60)
+    _, k, v = synth.make_qkv(2, Hkv, n, d, seed=61)
+    rows = np.arange(2 * H * n)
+    o, lse = oracle_mod.attn_rows_gqa(q, k, v, 0.3, causal, window, rows)
+    o_ref, lse_ref, _ = _brute_gqa(q, k, v, 0.3, causal, window)
+    np.testing.assert_allclose(o, o_ref.reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref.reshape(-1), rtol=0, atol=1e-12)
+
+
+def test_gqa_equals_multi_head_with_repeated_kv(oracle_mod):
+    """MQA/GQA is multi-head attention whose K/V heads are repeated within each
+    group of H/Hkv consecutive query heads (not interleaved across groups)."""
+    B, H, Hkv, n, d = 2, 8, 2, 50, 32
+    q, _, _ = synth.make_qkv(B, H, n, d, seed=62)
+    _, k, v = synth.make_qkv(B, Hkv, n, d, seed=63)
+    rows = np.arange(B * H * n)
+    o, lse = oracle_mod.attn_rows_gqa(q, k, v, 0.2, True, -1, rows)
+    kr = k.repeat_interleave(H // Hkv, dim=1).contiguous()
+    vr = v.repeat_interleave(H // Hkv, dim=1).contiguous()
+    o_m, lse_m, _ = oracle_mod.attn_rows(q, kr, vr, 0.2, True, -1, rows)
+    assert np.array_equal(o, o_m) and np.array_equal(lse, lse_m)
+    # the other plausible mapping (h % Hkv) gives a different answer
+    kw = k.repeat(1, H // Hkv, 1, 1).contiguous()
+    vw = v.repeat(1, H // Hkv, 1, 1).contiguous()
+    o_w, _, _ = oracle_mod.attn_rows(q, kw, vw, 0.2, True, -1, rows)
+    assert not np.allclose(o, o_w)
+
+
+def test_gqa_rejects_non_dividing_heads(oracle_mod):
+    q, _, _ = synth.make_qkv(1, 4, 8, 16)
+    _, k, v = synth.make_qkv(1, 3, 8, 16)
+    with pytest.raises(ValueError):
+        oracle_mod.attn_rows_gqa(q, k, v, 0.25, False, -1, [0])
