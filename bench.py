@@ -188,12 +188,12 @@ def cpu_baseline_leg(wl, o_gpu=None, lse_gpu=None, target_s: float = 15.0):
     # calibrate on a small sample, then size the sample to ~target_s seconds
     probe = torch.randint(0, total, (64,), generator=g).numpy()
     t0 = time.perf_counter()
-    oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe)
     dt = max(time.perf_counter() - t0, 1e-3)
     nrows = int(min(total, max(64, 64 * target_s / dt)))
     rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
     t0 = time.perf_counter()
-    o_ref, lse_ref, _ = oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, rows)
+    o_ref, lse_ref = oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, rows)
     dt = time.perf_counter() - t0
     out = {"value": nrows * flops_per_row / dt / 1e12, "unit": "TFLOP/s",
            "cores": oracle.num_threads(), "kind": "oracle",
@@ -229,17 +229,17 @@ def run_reference(args, wl, world, rank):
     # each step: a bounded sample sized so warmup + steps stay within ~2 minutes
     probe = torch.randint(0, total, (32,), generator=g).numpy()
     t0 = time.perf_counter()
-    oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe)
     per_row = max((time.perf_counter() - t0) / 32, 1e-6)
     budget = 120.0 / max(1, args.steps + args.warmup)
     nrows = int(max(8, min(total, budget / per_row)))
     samples = [np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
                for _ in range(args.steps + args.warmup)]
     for i in range(args.warmup):
-        oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, samples[i])
+        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[i])
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, samples[args.warmup + i])
+        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[args.warmup + i])
     dt = time.perf_counter() - t0
     value = args.steps * nrows * flops_per_row / dt / 1e12
     sample = f"{nrows} random query rows per step (seed 3) of {wl.name}, fp64 oracle"
@@ -255,6 +255,37 @@ def run_reference(args, wl, world, rank):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_e2e(args, wl, q, k, v, o, lse, flops, dev, stream, world):
+    """The metric through the host-buffer C-ABI entry point: pinned host
+    inputs copied in, kernel, O and LSE copied out, all inside the timed
+    region, every step."""
+    import exact_softmax_attention_04_b200 as attn
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    lh = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
+           "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
+    attn.host_staging_release()
+
+    return e2e
 
 
 def run_ours(args, wl, world, rank, local):
@@ -314,42 +345,36 @@ def run_ours(args, wl, world, rank, local):
         return 0
 
     # end to end through the host-buffer entry point: H2D of q,k,v, kernel,
-    # D2H of o and lse, every step
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    oh = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
-    lh = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, pin_memory=True)
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        attn.attn_fwd_host(qh, kh, vh, wl.scale, wl.causal, wl.window, out=oh, lse=lh, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    st = attn.sync_status(stream)
-    if st != attn.ATTN_OK:
-        raise RuntimeError(attn.strerror(st))
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e = {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-           "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
-           "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
-    attn.host_staging_release()
+    # D2H of o and lse, every step (that entry point takes equal head counts)
+    e2e = None
+    if wl.kv_heads == wl.H:
+        e2e = run_e2e(args, wl, q, k, v, o, lse, flops, dev, stream, world)
+    else:
+        e2e = {"value": None, "unit": "TFLOP/s",
+               "note": "grouped-query workload: the host-buffer entry point takes equal head counts"}
 
     traffic = recorded_traffic(wl.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
                 "frac": achieved / bf16_peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "algorithmic_flops_per_launch": flops,
-                "min_hbm_bytes_per_launch": 4 * q.numel() * 2 + lse.numel() * 4,
+                "min_hbm_bytes_per_launch": 2 * q.numel() * 2 + 2 * k.numel() * 2 + lse.numel() * 4,
                 "kernel_ms_per_launch": per_launch_ms}
     if traffic is not None:
         roofline["traffic_gbs"] = traffic / (per_launch_ms / 1e3) / 1e9
 
     if rank != 0:
         return 0
+    in_bytes = q.numel() * 2 + 2 * k.numel() * 2
+    sustained = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            sustained = float(json.load(fh)["bf16_tflops_sustained"])
+    except (OSError, KeyError, ValueError):
+        pass
+    if sustained:
+        roofline["frac_of_sustained_peak"] = achieved / sustained
+        roofline["sustained_peak"] = sustained
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -357,9 +382,9 @@ def run_ours(args, wl, world, rank, local):
         "data": "synthetic",
         "config": {**wl.describe(), "global_batch": wl.B * world, "seq_len": wl.n,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"no flush: inputs {3 * q.numel() * 2 / 1e6:.0f} MB + outputs "
+                   "l2": f"no flush: inputs {in_bytes / 1e6:.0f} MB + outputs "
                          f"{(o.numel() * 2 + lse.numel() * 4) / 1e6:.0f} MB per step "
-                         + ("exceed" if 3 * q.numel() * 2 > 126e6 else "do NOT exceed") + " the 126 MB L2"},
+                         + ("exceed" if in_bytes > 126e6 else "do NOT exceed") + " the 126 MB L2"},
         "pct_of_peak": 100.0 * value / world / bf16_peak,
         "roofline": roofline,
         "e2e": e2e,
@@ -381,7 +406,8 @@ def run_sweep(args):
     from exact_softmax_attention_04_b200 import synth
     torch.cuda.set_device(0)
     bf16_peak, hbm_peak, peak_src = peaks()
-    wls = [synth.SMALL_CAUSAL, synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072] + synth.sweep()
+    wls = [synth.SMALL_CAUSAL, synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072,
+           synth.GQA_N8192] + synth.sweep()
     for wl in wls:
         q, k, v = synth.make_inputs(wl)
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()

@@ -27,8 +27,8 @@ ATTN_ERR_TIMEOUT = 4
 ATTN_ERR_TOO_LARGE = 5
 
 # Every symbol include/attn.h declares.
-EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_host_staging_release", "attn_sync_status",
-           "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc")
+EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_release",
+           "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc")
 
 
 class AttnError(RuntimeError):
@@ -52,6 +52,8 @@ def load_library(path: str) -> ctypes.CDLL:
     fwd_args = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
     lib.attn_fwd.argtypes = fwd_args
     lib.attn_fwd.restype = i
+    lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd_gqa.restype = i
     lib.attn_fwd_host.argtypes = fwd_args
     lib.attn_fwd_host.restype = i
     lib.attn_fwd_host_noalloc.argtypes = fwd_args
@@ -94,7 +96,8 @@ def _stream_handle(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
     return s.cuda_stream
 
 
-def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device: bool) -> None:
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device: bool,
+               grouped: bool = False) -> None:
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16:
             raise TypeError(f"{name} must be bf16")
@@ -106,7 +109,11 @@ def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device: bool) 
             raise ValueError(f"{name} must be a CUDA tensor")
         if not device and t.is_cuda:
             raise ValueError(f"{name} must be a host tensor")
-    if not (q.shape == k.shape == v.shape):
+    if grouped:
+        if not (k.shape == v.shape and k.shape[0] == q.shape[0] and k.shape[2:] == q.shape[2:]
+                and q.shape[1] % k.shape[1] == 0):
+            raise ValueError("k and v must be [B, Hkv, n, d] with Hkv dividing H")
+    elif not (q.shape == k.shape == v.shape):
         raise ValueError("q, k and v must have the same shape")
     if device and not (q.device == k.device == v.device):
         raise ValueError("q, k and v must be on one device")
@@ -118,12 +125,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
              ) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T) V and its per-row log-sum-exp, on the GPU.
 
-    q, k, v: bf16 CUDA tensors [B, H, n, d], contiguous, d in {64, 128}.
+    q: bf16 CUDA tensor [B, H, n, d]; k, v: [B, H, n, d], or [B, Hkv, n, d]
+    with Hkv dividing H for grouped-query / multi-query attention (query
+    head h reads key/value head h // (H // Hkv)). Contiguous, d in {64, 128}.
     causal / window: see include/attn.h (window >= 0 needs causal).
     Returns (o bf16 [B, H, n, d], lse fp32 [B, H, n]); enqueued on ``stream``
     (default: the current stream), asynchronous like any CUDA op.
     """
-    _check_qkv(q, k, v, device=True)
+    grouped = k.dim() == 4 and q.dim() == 4 and k.shape[1] != q.shape[1]
+    _check_qkv(q, k, v, device=True, grouped=grouped)
     B, H, n, d = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -136,11 +146,16 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     if lse.shape != (B, H, n) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 tensor [B, H, n]")
     with torch.cuda.device(q.device):
-        rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                           B, H, n, d, float(scale), int(bool(causal)), int(window),
-                           _stream_handle(stream))
+        if grouped:
+            rc = lib().attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, H, k.shape[1], n, d, float(scale),
+                                    int(bool(causal)), int(window), _stream_handle(stream))
+        else:
+            rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, H, n, d, float(scale), int(bool(causal)),
+                                int(window), _stream_handle(stream))
     if rc != ATTN_OK:
-        raise AttnError(rc, "attn_fwd")
+        raise AttnError(rc, "attn_fwd_gqa" if grouped else "attn_fwd")
     return out, lse
 
 

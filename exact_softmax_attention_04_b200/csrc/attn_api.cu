@@ -80,10 +80,12 @@ bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const vo
 }
 
 int check_args(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
-               int H, int n, int d, float scale, int causal, int window, bool device_buffers)
+               int H, int n, int d, float scale, int causal, int window, bool device_buffers,
+               int Hkv = -1)
 {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
     if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return ATTN_ERR_INVALID;
+    if (Hkv != -1 && (Hkv <= 0 || H % Hkv != 0)) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
     if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
     const int64_t bh = static_cast<int64_t>(B) * H;
@@ -102,15 +104,18 @@ int check_args(const void *q, const void *k, const void *v, const void *o, const
 
 template <int D>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int n,
-               float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+               float scale, int causal, int window, cudaStream_t stream, int dev, int *status,
+               int Hkv = -1)
 {
     using Cfg = attn_sm100::FwdCfg<D>;
     auto enc = encoder();
     if (!enc) return ATTN_ERR_CUDA;
+    if (Hkv < 0) Hkv = H;
     const int64_t bh = static_cast<int64_t>(B) * H;
+    const int64_t bhkv = static_cast<int64_t>(B) * Hkv;
     CUtensorMap mq, mk, mv, mo;
-    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
-        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mo, o, bh, n, D))
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bhkv, n, D) ||
+        !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mo, o, bh, n, D))
         return ATTN_ERR_CUDA;
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -134,6 +139,8 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     attn_sm100::FwdParams p;
     p.lse = lse;
     p.status = status;
+    p.heads = H;
+    p.kv_heads = Hkv;
     p.n = n;
     p.num_q_tiles = (n + attn_sm100::BM - 1) / attn_sm100::BM;
     p.num_cta_tiles = (p.num_q_tiles + attn_sm100::QT - 1) / attn_sm100::QT;
@@ -159,6 +166,22 @@ extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, fl
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (d == 64) return launch_fwd<64>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status);
     return launch_fwd<128>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status);
+}
+
+extern "C" int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                            int H, int Hkv, int n, int d, float scale, int causal, int window,
+                            void *stream)
+{
+    const int rc = check_args(q, k, v, o, lse, B, H, n, d, scale, causal, window, true, Hkv);
+    if (rc != ATTN_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    int *status = status_word(dev);
+    if (!status) return ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return launch_fwd<64>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status, Hkv);
+    return launch_fwd<128>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status, Hkv);
 }
 
 extern "C" int attn_fwd_host(const void *q, const void *k, const void *v, void *o, float *lse, int B,

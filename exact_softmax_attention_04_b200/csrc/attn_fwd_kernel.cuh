@@ -1,7 +1,10 @@
 // attn_fwd_kernel.cuh - exact softmax attention forward for sm_100a.
 //
 // One CTA computes two adjacent 128-row query tiles Q_0, Q_1 (256 rows) of
-// one (batch, head). For each key/value tile j allowed by the mask:
+// one (batch, query head); its keys and values come from the key/value head
+// of that query head's group (grouped-query attention; one K/V head per
+// query head in the multi-head case). For each key/value tile j allowed by
+// the mask:
 //   S_s = Q_s K_j^T                     (tcgen05 MMA, smem x smem -> TMEM fp32)
 //   online softmax on S_s, row by row   (running max m, running normaliser l)
 //   O_s += P_s V_j                      (tcgen05 MMA, P from TMEM x V from smem)
@@ -71,6 +74,8 @@ constexpr int STATUS_WAIT_TIMEOUT = 1;
 struct FwdParams {
     float *lse;        // [B*H, n]
     int *status;       // device status word
+    int heads;         // H: query heads per batch
+    int kv_heads;      // H_kv: key/value heads per batch (divides H)
     int n;
     int num_q_tiles;   // ceil(n / BM)
     int num_cta_tiles; // ceil(num_q_tiles / QT)
@@ -228,6 +233,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     // L2); within a head the late pairs (the most expensive under a causal
     // mask) start first.
     const int bh = blockIdx.x / p.num_cta_tiles;
+    // Grouped-query attention: query head h of batch b reads key/value head
+    // h / (H / H_kv) of that batch (H_kv = H: one K/V head per query head).
+    const int bkv = (bh / p.heads) * p.kv_heads + (bh % p.heads) / (p.heads / p.kv_heads);
     const int ct = p.num_cta_tiles - 1 - static_cast<int>(blockIdx.x % p.num_cta_tiles);
     const int m0 = ct * (QT * BM);
     const int n = p.n;
@@ -313,7 +321,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             const int k0 = (jlo + i / 2) * BN;
 #pragma unroll
             for (int b = 0; b < C::BOXES; ++b)
-                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
+                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bkv);
             ++issued;
         }
         if (issued < 2 * nkv) {

@@ -35,10 +35,15 @@ class Workload:
     window: int = -1  # < 0: no window; >= 0: keys max(0, i - window) .. i
     q_std: float = 1.0
     seed: int = 0
+    Hkv: int = 0      # key/value heads (grouped-query attention); 0 means H
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv if self.Hkv > 0 else self.H
 
     @property
     def mask(self) -> str:
@@ -51,6 +56,7 @@ class Workload:
             "workload": self.name,
             "B": self.B,
             "H": self.H,
+            "H_kv": self.kv_heads,
             "n": self.n,
             "d": self.d,
             "mask": self.mask,
@@ -77,28 +83,29 @@ def attended_pairs_per_head(n: int, causal: bool, window: int) -> int:
     return n * n
 
 
-def unmasked_flops(wl: Workload) -> int:
+def unmasked_flops(wl: "Workload") -> int:
     """4*d FLOPs per attended pair (2*d for QK^T, 2*d for PV), times B*H."""
     return 4 * wl.d * attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H
 
 
-def make_qkv(B: int, H: int, n: int, d: int, seed: int = 0, q_std: float = 1.0
+def make_qkv(B: int, H: int, n: int, d: int, seed: int = 0, q_std: float = 1.0, Hkv: int = 0
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Q, K, V as contiguous bf16 CPU tensors [B, H, n, d] (recipe above)."""
+    """Q as a contiguous bf16 CPU tensor [B, H, n, d] and K, V as [B, Hkv, n, d]
+    (Hkv = H when 0), following the recipe above."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
-    shape = (B, H, n, d)
-    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    q = torch.randn((B, H, n, d), generator=g, dtype=torch.float32)
     if q_std != 1.0:
         q.mul_(q_std)
     q = q.to(torch.bfloat16)
-    k = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
-    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kv_shape = (B, Hkv if Hkv > 0 else H, n, d)
+    k = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
 def make_inputs(wl: Workload):
-    return make_qkv(wl.B, wl.H, wl.n, wl.d, wl.seed, wl.q_std)
+    return make_qkv(wl.B, wl.H, wl.n, wl.d, wl.seed, wl.q_std, wl.Hkv)
 
 
 def sample_rows(B: int, H: int, n: int, per_head_random: int = 256, seed: int = 1,
@@ -127,6 +134,9 @@ SMALL_CAUSAL = Workload("B1-H2-n256-d64-causal", 1, 2, 256, 64, True)
 FULL_N8192 = Workload("B8-H8-n8192-d64-none", 8, 8, 8192, 64, False)
 WINDOW_N32768 = Workload("B1-H32-n32768-d128-window4096", 1, 32, 32768, 128, True, 4096)
 CAUSAL_N131072 = Workload("B1-H8-n131072-d128-causal", 1, 8, 131072, 128, True)
+# Grouped-query attention with the head layout the pages quote for LLaMA-2 70B
+# (64 query heads sharing 8 key/value heads), causal, 8192 tokens.
+GQA_N8192 = Workload("B1-H64-Hkv8-n8192-d128-causal", 1, 64, 8192, 128, True, Hkv=8)
 
 
 def sweep() -> List[Workload]:
@@ -143,7 +153,7 @@ def sweep() -> List[Workload]:
 
 
 def by_name(name: str) -> Optional[Workload]:
-    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072] + sweep():
+    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072, GQA_N8192] + sweep():
         if wl.name == name:
             return wl
     return None

@@ -91,6 +91,24 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
              void *stream);
 
 /*
+ * attn_fwd_gqa - grouped-query (and multi-query) attention on device buffers.
+ *
+ * Grouped-query attention ("week17 efficiency attention", MQA / GQA section):
+ * G = Hkv groups of query heads share one key/value head; Hkv = 1 is
+ * multi-query attention, Hkv = H is attn_fwd.
+ *
+ *   q, o    : device, bf16 [B, H, n, d]
+ *   k, v    : device, bf16 [B, Hkv, n, d]
+ *   lse     : device, fp32 [B, H, n]
+ *   Hkv     : >= 1 and divides H (else ATTN_ERR_INVALID); query head h reads
+ *             key/value head h / (H / Hkv)
+ * Everything else (alignment, d, scale, masks, stream, errors) as attn_fwd.
+ */
+ATTN_API int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int H, int Hkv, int n, int d, float scale, int causal,
+                          int window, void *stream);
+
+/*
  * attn_fwd_host - the same operation on HOST buffers, copies included.
  *
  *   q, k, v : host, bf16 [B, H, n, d] (pinned memory makes the copies async)

@@ -73,6 +73,8 @@ def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
               ) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
     """O (nrows x d), LSE (nrows) and optionally weights (nrows x n) for flat rows."""
     lib = _load()
+    if not (q.shape == k.shape == v.shape) or len(q.shape) != 4:
+        raise ValueError("q, k and v must all be [B, H, n, d] (see attn_rows_gqa for fewer K/V heads)")
     B, H, n, d = q.shape
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
@@ -113,6 +115,8 @@ def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1
              ) -> Tuple[np.ndarray, np.ndarray]:
     """Full O [B,H,n,d] and LSE [B,H,n] in fp64."""
     lib = _load()
+    if not (q.shape == k.shape == v.shape) or len(q.shape) != 4:
+        raise ValueError("q, k and v must all be [B, H, n, d]")
     B, H, n, d = q.shape
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     o = np.empty((B, H, n, d), dtype=np.float64)

@@ -111,3 +111,22 @@ def test_missing_library_fails_loudly(monkeypatch, attn):
     monkeypatch.setattr(pkg, "LIB_PATH", "/nonexistent/libattn_b200.so")
     with pytest.raises(ImportError):
         pkg._load()
+
+
+def test_gqa_entry_point_rejects_bad_head_counts(attn):
+    lib = attn.lib()
+    for Hkv in (0, -2, 3, 16):
+        rc = lib.attn_fwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, Hkv, 128, 64, 0.125, 1, -1, None)
+        assert rc == attn.ATTN_ERR_INVALID, Hkv
+    rc = lib.attn_fwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, 128, 80, 0.125, 1, -1, None)
+    assert rc == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_binding_checks_grouped_shapes(attn):
+    import torch
+    q = torch.zeros(1, 8, 16, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 3, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn._check_qkv(q, kv, kv, device=False, grouped=True)
+    kv2 = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    attn._check_qkv(q, kv2, kv2, device=False, grouped=True)

@@ -271,6 +271,10 @@ def test_oracle_rejects_bad_arguments(oracle_mod):
         oracle_mod.attn_fwd(q, k, v, 0.25, False, 3)  # window needs causal
     with pytest.raises(ValueError):
         oracle_mod.attn_rows(q, k, v, 0.25, True, -1, [8])  # row out of range
+    _, k2, v2 = synth.make_qkv(1, 1, 8, 16, Hkv=1)
+    q2, _, _ = synth.make_qkv(1, 2, 8, 16)
+    with pytest.raises(ValueError):
+        oracle_mod.attn_rows(q2, k2, v2, 0.25, True, -1, [0])  # fewer K/V heads: use attn_rows_gqa
 
 
 def test_pair_count_matches_explicit_masks(oracle_mod):

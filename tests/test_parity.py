@@ -147,3 +147,44 @@ def test_full_size_workloads_sampled(attn, oracle_mod, wl):
     q, k, v = synth.make_inputs(wl)
     o2, l2 = _gpu(attn, q, k, v, wl.causal, wl.window, wl.scale)
     assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 3), (8, 1)])
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 100)])
+def test_gqa_small_shapes_in_full(attn, oracle_mod, d, H, Hkv, causal, window):
+    n = 300
+    q, k, v = synth.make_qkv(2, H, n, d, seed=H * 10 + Hkv, q_std=2.0, Hkv=Hkv)
+    sc = 1.0 / np.sqrt(d)
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), sc, causal, window)
+    assert attn.sync_status() == attn.ATTN_OK
+    rows = np.arange(2 * H * n)
+    o_ref, lse_ref = oracle_mod.attn_rows_gqa(q, k, v, sc, causal, window, rows)
+    assert_close(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), o_ref, lse_ref,
+                 f"gqa H{H} Hkv{Hkv} d{d} c{causal} w{window}")
+
+
+def test_gqa_equals_multi_head_on_repeated_kv_bit_for_bit(attn):
+    B, H, Hkv, n, d = 2, 8, 2, 777, 128
+    q, k, v = synth.make_qkv(B, H, n, d, seed=70, Hkv=Hkv)
+    o_g, l_g = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), None, True, -1)
+    kr = k.repeat_interleave(H // Hkv, dim=1).contiguous().cuda()
+    vr = v.repeat_interleave(H // Hkv, dim=1).contiguous().cuda()
+    o_m, l_m = attn.attn_fwd(q.cuda(), kr, vr, None, True, -1)
+    assert attn.sync_status() == attn.ATTN_OK
+    assert torch.equal(o_g, o_m) and torch.equal(l_g, l_m)
+
+
+def test_gqa_workload_sampled(attn, oracle_mod):
+    wl = synth.GQA_N8192
+    q, k, v = synth.make_inputs(wl)
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), wl.scale, wl.causal, wl.window)
+    assert attn.sync_status() == attn.ATTN_OK
+    rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=8, bound_every=16, edge=8)
+    idx = torch.as_tensor(rows, device=o.device)
+    o_s = o.view(-1, wl.d)[idx].float().cpu().numpy()
+    l_s = lse.view(-1)[idx].cpu().numpy()
+    o_ref, lse_ref = oracle_mod.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, rows)
+    assert_close(o_s, l_s, o_ref, lse_ref, wl.name)
