@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for exact softmax attention (test infrastructure only).
+"""fp64 CPU oracle for exact softmax attention, forward and backward (test
+infrastructure only).
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package. The CUDA product path never does.
@@ -54,6 +55,9 @@ def _load():
         lib.oracle_matmul_f64.restype = ip
         lib.oracle_mask_row.argtypes = [i64, i64, ip, i64, vp]
         lib.oracle_mask_row.restype = ip
+        lib.oracle_attn_bwd_rows_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
+                                                 i64, vp, i64, vp, i64, vp, vp, vp]
+        lib.oracle_attn_bwd_rows_f64.restype = ip
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ip
         _lib = lib
@@ -127,6 +131,60 @@ def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd_f64 rejected its arguments (rc={rc})")
     return o, lse
+
+
+IN_BF16 = 0
+IN_F64 = 1
+
+
+def _bwd_input(t):
+    """(array, type) for the backward oracle: bf16 torch tensors as their bit
+    patterns, anything else as contiguous fp64."""
+    import torch
+    if isinstance(t, torch.Tensor) and t.dtype == torch.bfloat16:
+        return _bits(t), IN_BF16
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.float64)), IN_F64
+
+
+def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=()
+                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Backward pass for selected rows. q, k, v, dout: [B, H, n, d], all bf16
+    torch tensors or all fp64 arrays. Returns dQ for the flat query rows
+    ``qrows`` (len x d) and dK, dV for the flat key rows ``krows`` (len x d
+    each), flat row = (b*H + h)*n + i, all fp64."""
+    lib = _load()
+    shapes = {tuple(x.shape) for x in (q, k, v, dout)}
+    if len(shapes) != 1 or len(q.shape) != 4:
+        raise ValueError("q, k, v and dout must all be [B, H, n, d]")
+    B, H, n, d = q.shape
+    ins = [_bwd_input(x) for x in (q, k, v, dout)]
+    if len({t for _, t in ins}) != 1:
+        raise TypeError("q, k, v and dout must be all bf16 or all floating point")
+    typ = ins[0][1]
+    qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64).reshape(-1))
+    kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64).reshape(-1))
+    dq = np.empty((qr.size, d), dtype=np.float64)
+    dk = np.empty((kr.size, d), dtype=np.float64)
+    dv = np.empty((kr.size, d), dtype=np.float64)
+    rc = lib.oracle_attn_bwd_rows_f64(ins[0][0].ctypes.data, ins[1][0].ctypes.data,
+                                      ins[2][0].ctypes.data, ins[3][0].ctypes.data, typ,
+                                      B, H, n, d, float(scale), int(bool(causal)), int(window),
+                                      qr.ctypes.data, qr.size, kr.ctypes.data, kr.size,
+                                      dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_rows_f64 rejected its arguments (rc={rc})")
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, window: int = -1
+             ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Full dQ, dK, dV [B, H, n, d] in fp64."""
+    B, H, n, d = q.shape
+    rows = np.arange(B * H * n, dtype=np.int64)
+    dq, dk, dv = attn_bwd_rows(q, k, v, dout, scale, causal, window, rows, rows)
+    return dq.reshape(B, H, n, d), dk.reshape(B, H, n, d), dv.reshape(B, H, n, d)
 
 
 def matmul(a: np.ndarray, b: np.ndarray, ta: bool = False, tb: bool = False) -> np.ndarray:

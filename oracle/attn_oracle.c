@@ -1,5 +1,6 @@
 /*
- * Exact scaled dot-product attention, forward pass: the fp64 CPU oracle.
+ * Exact scaled dot-product attention, forward and backward passes: the fp64
+ * CPU oracle.
  *
  * TEST INFRASTRUCTURE ONLY. This file is the checker of the CUDA path, not
  * part of it. Only the test suite, the smoke check and the benchmark's CPU
@@ -80,7 +81,7 @@ double oracle_dot_f64(const double *a, int64_t sa, const double *b, int64_t sb, 
 int oracle_matmul_f64(int64_t m, int64_t n, int64_t k, const double *A, int ta,
                       const double *B, int tb, double *C)
 {
-    if (m < 0 || n < 0 || k < 0 || (!A && m * k) || (!B && k * n) || (!C && m * n))
+    if (m < 0 || n < 0 || k < 0 || (!A && m * k != 0) || (!B && k * n != 0) || (!C && m * n != 0))
         return 1;
     for (int64_t i = 0; i < m; ++i) {
         const double *arow = ta ? A + i : A + i * k;
@@ -262,4 +263,214 @@ int oracle_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ========================================================================
+ * Backward pass: gradients of the attention output with respect to Q, K, V.
+ *
+ * The pages note that FlashAttention recomputes in the backward pass what it
+ * needs instead of storing the score matrix ("Efficient Transformers ...",
+ * section "Family 3"). What the backward pass computes is fixed by the
+ * forward definition above and the chain rule alone: for an upstream
+ * gradient dO = dL/dO, with P_ij = exp(s_ij - LSE_i) for j in A(i) (0
+ * elsewhere) and s_ij = scale * q_i . k_j,
+ *
+ *   dV_j  = sum_i P_ij dO_i                          (O_i = sum_j P_ij v_j)
+ *   dP_ij = dO_i . v_j
+ *   dS_ij = P_ij (dP_ij - sum_t P_it dP_it)          (Jacobian of a row softmax)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i
+ *
+ * The row term sum_t P_it dP_it is computed as written, from the row's own
+ * weights (not from O). Every sum runs over the allowed (i, j) pairs only.
+ * Rows are independent for dQ; a key row j needs, for every query i that
+ * attends to it, that query's LSE_i and row term, so those are computed for
+ * all rows of each head that a requested key row belongs to.
+ *
+ * Inputs are Q, K, V, dO as [B, H, n, d], either bf16 bit patterns
+ * (ORACLE_IN_BF16) or fp64 values (ORACLE_IN_F64); all arithmetic is fp64.
+ * ======================================================================== */
+
+#define ORACLE_IN_BF16 0
+#define ORACLE_IN_F64 1
+
+static double in_at(const void *p, int type, int64_t idx)
+{
+    return type == ORACLE_IN_F64 ? ((const double *)p)[idx] : bf16_to_f64(((const uint16_t *)p)[idx]);
+}
+
+/* One query row's softmax statistics and, if dq != NULL, its gradient.
+ * base = (b*H + h)*n*d is the head's offset; s and w are n-long scratch. */
+static void bwd_row(const void *q, const void *k, const void *v, const void *dout, int type,
+                    int64_t base, int64_t n, int64_t d, double scale, int causal, int64_t window,
+                    int64_t i, unsigned char *allowed, double *s, double *dp,
+                    double *lse_out, double *rowterm_out, double *dq)
+{
+    oracle_mask_row(n, i, causal, window, allowed);
+    double M = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+        if (!allowed[j])
+            continue;
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            acc += in_at(q, type, base + i * d + c) * in_at(k, type, base + j * d + c);
+        s[j] = scale * acc;
+        if (s[j] > M)
+            M = s[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < n; ++j)
+        if (allowed[j])
+            Z += exp(s[j] - M);
+    const double lse = M + log(Z);
+    /* dP_ij and the row term sum_j P_ij dP_ij */
+    double rowterm = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        if (!allowed[j])
+            continue;
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            acc += in_at(dout, type, base + i * d + c) * in_at(v, type, base + j * d + c);
+        dp[j] = acc;
+        rowterm += exp(s[j] - lse) * acc;
+    }
+    if (lse_out)
+        *lse_out = lse;
+    if (rowterm_out)
+        *rowterm_out = rowterm;
+    if (dq) {
+        for (int64_t c = 0; c < d; ++c)
+            dq[c] = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            if (!allowed[j])
+                continue;
+            const double ds = exp(s[j] - lse) * (dp[j] - rowterm);
+            for (int64_t c = 0; c < d; ++c)
+                dq[c] += ds * in_at(k, type, base + j * d + c);
+        }
+        for (int64_t c = 0; c < d; ++c)
+            dq[c] *= scale;
+    }
+}
+
+/*
+ * Gradients for selected rows.
+ *   q, k, v, dout : [B, H, n, d] inputs of element type `type`
+ *   qrows (nq)    : flat query rows (b*H + h)*n + i whose dQ is wanted -> dq (nq x d)
+ *   krows (nk)    : flat key rows (b*H + h)*n + j whose dK, dV are wanted
+ *                   -> dk, dv (nk x d each)
+ * window >= 0 requires causal. Returns 0 on success, nonzero on bad input.
+ */
+int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const void *dout, int type,
+                             int64_t B, int64_t H, int64_t n, int64_t d, double scale, int causal,
+                             int64_t window, const int64_t *qrows, int64_t nq, const int64_t *krows,
+                             int64_t nk, double *dq, double *dk, double *dv)
+{
+    if (!q || !k || !v || !dout || B <= 0 || H <= 0 || n <= 0 || d <= 0)
+        return 1;
+    if (type != ORACLE_IN_BF16 && type != ORACLE_IN_F64)
+        return 1;
+    if (window >= 0 && !causal)
+        return 1;
+    if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv)) || nq < 0 || nk < 0)
+        return 1;
+    const int64_t rows_total = B * H * n;
+    for (int64_t r = 0; r < nq; ++r)
+        if (qrows[r] < 0 || qrows[r] >= rows_total)
+            return 1;
+    for (int64_t r = 0; r < nk; ++r)
+        if (krows[r] < 0 || krows[r] >= rows_total)
+            return 1;
+
+    /* heads that requested key rows belong to, and their per-row statistics */
+    const int64_t nheads = B * H;
+    int64_t *slot = (int64_t *)malloc(sizeof(int64_t) * (size_t)nheads);
+    if (!slot)
+        return 2;
+    for (int64_t h = 0; h < nheads; ++h)
+        slot[h] = -1;
+    int64_t nstat = 0;
+    for (int64_t r = 0; r < nk; ++r)
+        if (slot[krows[r] / n] < 0)
+            slot[krows[r] / n] = nstat++;
+    int64_t *stat_head = (int64_t *)malloc(sizeof(int64_t) * (size_t)(nstat + 1));
+    double *lse = (double *)malloc(sizeof(double) * (size_t)(nstat * n + 1));
+    double *rowterm = (double *)malloc(sizeof(double) * (size_t)(nstat * n + 1));
+    if (!stat_head || !lse || !rowterm) {
+        free(slot);
+        free(stat_head);
+        free(lse);
+        free(rowterm);
+        return 2;
+    }
+    for (int64_t h = 0; h < nheads; ++h)
+        if (slot[h] >= 0)
+            stat_head[slot[h]] = h;
+
+    int bad = 0;
+#pragma omp parallel
+    {
+        unsigned char *allowed = (unsigned char *)malloc((size_t)n);
+        double *s = (double *)malloc(sizeof(double) * (size_t)n);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)n);
+        if (!allowed || !s || !dp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            /* 1. statistics of every row of the heads with requested key rows */
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t t = 0; t < nstat * n; ++t) {
+                const int64_t h = stat_head[t / n], i = t % n;
+                bwd_row(q, k, v, dout, type, h * n * d, n, d, scale, causal, window, i, allowed, s,
+                        dp, &lse[t], &rowterm[t], NULL);
+            }
+            /* 2. dQ of the requested query rows */
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nq; ++r) {
+                const int64_t h = qrows[r] / n, i = qrows[r] % n;
+                bwd_row(q, k, v, dout, type, h * n * d, n, d, scale, causal, window, i, allowed, s,
+                        dp, NULL, NULL, dq + r * d);
+            }
+            /* 3. dK, dV of the requested key rows: sums over the queries that
+             * attend to key j, with each query's own LSE and row term */
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nk; ++r) {
+                const int64_t h = krows[r] / n, j = krows[r] % n;
+                const int64_t base = h * n * d;
+                const double *L = lse + slot[h] * n;
+                const double *R = rowterm + slot[h] * n;
+                double *gk = dk + r * d, *gv = dv + r * d;
+                for (int64_t c = 0; c < d; ++c)
+                    gk[c] = gv[c] = 0.0;
+                for (int64_t i = 0; i < n; ++i) {
+                    /* is key j in A(i)? */
+                    if (causal && j > i)
+                        continue;
+                    if (window >= 0 && j < i - window)
+                        continue;
+                    double sij = 0.0, dpij = 0.0;
+                    for (int64_t c = 0; c < d; ++c) {
+                        sij += in_at(q, type, base + i * d + c) * in_at(k, type, base + j * d + c);
+                        dpij += in_at(dout, type, base + i * d + c) * in_at(v, type, base + j * d + c);
+                    }
+                    const double pij = exp(scale * sij - L[i]);
+                    const double dsij = pij * (dpij - R[i]);
+                    for (int64_t c = 0; c < d; ++c) {
+                        gv[c] += pij * in_at(dout, type, base + i * d + c);
+                        gk[c] += dsij * in_at(q, type, base + i * d + c);
+                    }
+                }
+                for (int64_t c = 0; c < d; ++c)
+                    gk[c] *= scale;
+            }
+        }
+        free(allowed);
+        free(s);
+        free(dp);
+    }
+    free(slot);
+    free(stat_head);
+    free(lse);
+    free(rowterm);
+    return bad ? 2 : 0;
 }
