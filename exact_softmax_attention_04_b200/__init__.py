@@ -28,7 +28,8 @@ ATTN_ERR_TOO_LARGE = 5
 
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_release",
-           "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc")
+           "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
+           "attn_bwd", "attn_bwd_workspace_bytes")
 
 
 class AttnError(RuntimeError):
@@ -66,6 +67,11 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_strerror.restype = ctypes.c_char_p
     lib.attn_attended_pairs.argtypes = [i64, i, i64]
     lib.attn_attended_pairs.restype = i64
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                             i, i, i, i, f, i, i, vp]
+    lib.attn_bwd.restype = i
+    lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.attn_bwd_workspace_bytes.restype = i64
     return lib
 
 
@@ -157,6 +163,54 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_gqa" if grouped else "attn_fwd")
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, H: int, n: int, d: int) -> int:
+    r = int(lib().attn_bwd_workspace_bytes(int(B), int(H), int(n), int(d)))
+    if r < 0:
+        raise ValueError("unsupported or invalid shape for attn_bwd")
+    return r
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, scale: Optional[float] = None,
+             causal: bool = False, window: int = -1, workspace: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, dk, dv) of the attention forward pass on the GPU.
+
+    q, k, v, o, dout: bf16 CUDA tensors [B, H, n, d], contiguous; o and lse
+    are attn_fwd's outputs for q, k, v with the same scale and mask; dout is
+    the upstream gradient dL/dO. ``workspace`` (optional) is a uint8 CUDA
+    tensor of at least bwd_workspace_bytes(B, H, n, d) bytes. Enqueued on
+    ``stream`` (default: the current stream).
+    """
+    _check_qkv(q, k, v, device=True)
+    for name, t in (("o", o), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous() or \
+                t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q on q's device")
+    B, H, n, d = q.shape
+    if lse.shape != (B, H, n) or lse.dtype != torch.float32 or not lse.is_contiguous() or \
+            lse.device != q.device:
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, n] on q's device")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = bwd_workspace_bytes(B, H, n, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace.device != q.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on q's device")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    with torch.cuda.device(q.device):
+        rc = lib().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            B, H, n, d, float(scale), int(bool(causal)), int(window),
+                            _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,

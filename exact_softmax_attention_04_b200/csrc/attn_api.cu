@@ -13,22 +13,14 @@
 
 #include "attn.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_host.h"
 
-namespace {
-
-constexpr int kMaxDevices = 64;
+namespace attn_host {
 
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 bool g_encode_tried = false;
 int *g_status[kMaxDevices] = {};
-bool g_smem_set[kMaxDevices][2] = {};
-
-struct Staging {
-    void *buf = nullptr;
-    size_t cap = 0;
-};
-Staging g_staging[kMaxDevices];
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -47,7 +39,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder()
     return g_encode;
 }
 
-// Device status word for the current device, allocated once and zeroed.
 int *status_word(int dev)
 {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -63,8 +54,6 @@ int *status_word(int dev)
     return g_status[dev];
 }
 
-// [B*H, n, d] bf16 viewed as a 3-D tensor (d fastest), boxes of 64 x 128 x 1,
-// 128-byte swizzle; rows past n read as zero and are clipped on store.
 bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int64_t bh,
                  int64_t n, int64_t d)
 {
@@ -78,6 +67,26 @@ bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const vo
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+int current_device(int *dev)
+{
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+}  // namespace attn_host
+
+namespace {
+
+using namespace attn_host;
+
+bool g_smem_set[kMaxDevices][2] = {};
+
+struct Staging {
+    void *buf = nullptr;
+    size_t cap = 0;
+};
+Staging g_staging[kMaxDevices];
 
 int check_args(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
                int H, int n, int d, float scale, int causal, int window, bool device_buffers,
@@ -260,7 +269,8 @@ extern "C" int attn_sync_status(void *stream)
     if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
     if (h != 0) {
         if (cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
-        return ATTN_ERR_TIMEOUT;
+        // bit 1: a bounded wait expired; any other bit: a kernel refused to run
+        return (h & attn_sm100::STATUS_WAIT_TIMEOUT) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
     }
     return ATTN_OK;
 }

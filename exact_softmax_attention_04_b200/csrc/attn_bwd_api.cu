@@ -1,0 +1,160 @@
+// attn_bwd_api.cu - host side of the backward pass: argument checks, workspace
+// layout, TMA descriptors and the three launches. Contracts in include/attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "attn.h"
+#include "attn_bwd_kernel.cuh"
+#include "attn_host.h"
+
+namespace {
+
+using namespace attn_host;
+
+bool g_bwd_set[kMaxDevices][2] = {};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout: [dQ accumulator fp32 B*H*n*d | lse2 fp32 B*H*n_pad |
+// delta fp32 B*H*n_pad], each part starting on a 256-byte boundary.
+struct BwdWorkspace {
+    size_t acc_bytes, stat_bytes, total;
+};
+
+BwdWorkspace workspace_layout(int64_t bh, int64_t n, int64_t d)
+{
+    const int64_t n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
+    BwdWorkspace w;
+    w.acc_bytes = round256(static_cast<size_t>(bh * n * d) * 4);
+    w.stat_bytes = round256(static_cast<size_t>(bh * n_pad) * 4);
+    w.total = w.acc_bytes + 2 * w.stat_bytes;
+    return w;
+}
+
+int check_bwd_args(int B, int H, int n, int d, float scale, int causal, int window)
+{
+    if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return ATTN_ERR_INVALID;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    if (bh > INT_MAX) return ATTN_ERR_INVALID;
+    // the fp32 accumulator (4 bytes per element) must be addressable
+    if (bh * n > INT64_MAX / (4 * static_cast<int64_t>(d) + 16)) return ATTN_ERR_INVALID;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (window >= 0 && !causal) return ATTN_ERR_UNSUPPORTED;
+    if (n > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
+    const int64_t ktiles = bh * ((n + attn_sm100::BN - 1) / attn_sm100::BN);
+    if (ktiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+template <int D>
+int launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+               const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int n,
+               float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+{
+    using Cfg = attn_sm100::BwdCfg<D>;
+    auto enc = encoder();
+    if (!enc) return ATTN_ERR_CUDA;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
+        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
+        !encode_bhnd(enc, &mdk, dk, bh, n, D) || !encode_bhnd(enc, &mdv, dv, bh, n, D))
+        return ATTN_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0];
+        if (!set) {
+            // Same rule as the forward kernel: the register split between
+            // warpgroups needs exactly the per-thread count it was computed for.
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, attn_sm100::attn_bwd_kernel<D>) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
+            if (cudaFuncSetAttribute(attn_sm100::attn_bwd_kernel<D>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM_BYTES) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+            set = true;
+        }
+    }
+    const BwdWorkspace w = workspace_layout(bh, n, D);
+    float *acc = reinterpret_cast<float *>(ws);
+    float *lse2 = reinterpret_cast<float *>(ws + w.acc_bytes);
+    float *delta = reinterpret_cast<float *>(ws + w.acc_bytes + w.stat_bytes);
+    const int n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
+
+    // 1. delta, lse2, zeroed accumulator
+    const int64_t prep_threads = bh * n_pad * (D / 8);
+    const int64_t prep_blocks = (prep_threads + 255) / 256;
+    if (prep_blocks > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    attn_sm100::attn_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, lse2, delta,
+        acc, bh, n, n_pad);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    // 2. main kernel
+    attn_sm100::BwdParams p;
+    p.dq_acc = acc;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.status = status;
+    p.n = n;
+    p.n_pad = n_pad;
+    p.num_k_tiles = (n + attn_sm100::BN - 1) / attn_sm100::BN;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal;
+    p.window = window < 0 ? -1 : window;
+    const unsigned grid = static_cast<unsigned>(bh * p.num_k_tiles);
+    attn_sm100::attn_bwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
+                                                                                    mdv, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    // 3. dQ accumulator -> bf16
+    const int64_t count8 = bh * n * D / 8;
+    const int64_t conv_blocks = (count8 + 255) / 256;
+    if (conv_blocks > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    attn_sm100::attn_bwd_dq_convert_kernel<<<static_cast<unsigned>(conv_blocks), 256, 0, stream>>>(
+        acc, static_cast<__nv_bfloat16 *>(dq), count8);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d)
+{
+    if (check_bwd_args(B, H, n, d, 1.f, 0, -1) != ATTN_OK) return -1;
+    return static_cast<int64_t>(workspace_layout(static_cast<int64_t>(B) * H, n, d).total);
+}
+
+extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                        const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                        size_t workspace_bytes, int B, int H, int n, int d, float scale, int causal,
+                        int window, void *stream)
+{
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
+    const int rc = check_bwd_args(B, H, n, d, scale, causal, window);
+    if (rc != ATTN_OK) return rc;
+    for (const void *ptr : {q, k, v, o, dout, static_cast<const void *>(dq), static_cast<const void *>(dk),
+                            static_cast<const void *>(dv), static_cast<const void *>(workspace)})
+        if (!aligned(ptr, 16)) return ATTN_ERR_INVALID;
+    if (!aligned(lse, 4)) return ATTN_ERR_INVALID;
+    if (workspace_bytes < workspace_layout(static_cast<int64_t>(B) * H, n, d).total) return ATTN_ERR_INVALID;
+    int dev = 0;
+    if (current_device(&dev) != ATTN_OK) return ATTN_ERR_CUDA;
+    int *status = status_word(dev);
+    if (!status) return ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    if (d == 64)
+        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window, st,
+                              dev, status);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window, st, dev,
+                           status);
+}

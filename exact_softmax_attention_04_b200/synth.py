@@ -104,6 +104,15 @@ def make_qkv(B: int, H: int, n: int, d: int, seed: int = 0, q_std: float = 1.0, 
     return q.contiguous(), k.contiguous(), v.contiguous()
 
 
+def make_dout(B: int, H: int, n: int, d: int, seed: int = 0) -> torch.Tensor:
+    """Upstream gradient dO for the backward pass: a contiguous bf16 CPU tensor
+    [B, H, n, d] of N(0, 1) draws from a CPU generator seeded seed + 1 (fp32
+    draws rounded to bf16)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 1)
+    return torch.randn((B, H, n, d), generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+
+
 def make_inputs(wl: Workload):
     return make_qkv(wl.B, wl.H, wl.n, wl.d, wl.seed, wl.q_std, wl.Hkv)
 

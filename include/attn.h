@@ -1,6 +1,6 @@
 /*
- * attn.h - C ABI of the B200 (sm_100a) exact softmax attention forward library
- * (libattn_b200.so).
+ * attn.h - C ABI of the B200 (sm_100a) exact softmax attention library
+ * (libattn_b200.so): forward pass, grouped-query forward, backward pass.
  *
  * The operation (all entry points that compute):
  *
@@ -46,6 +46,7 @@
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 /* Exported symbols of the shared library (everything else is hidden). */
@@ -162,10 +163,57 @@ ATTN_API int attn_fwd_host_noalloc(const void *q, const void *k, const void *v, 
                                    int causal, int window, void *stream);
 
 /*
+ * attn_bwd - enqueue the attention backward pass on device buffers.
+ *
+ * Gradients of a loss L with respect to Q, K and V given dO = dL/dO, for the
+ * forward pass of attn_fwd with the same mask and scale. The attention
+ * weights are recomputed from Q, K and the forward pass's LSE rather than
+ * stored (the recompute in the backward pass named in "Efficient
+ * Transformers: Sparse Attention, Linear Attention and FlashAttention",
+ * section "Family 3"). With P_ij = exp(scale * q_i . k_j - LSE_i) on the
+ * allowed pairs (0 elsewhere):
+ *
+ *   dV_j = sum_i P_ij dO_i
+ *   dS_ij = P_ij (dO_i . v_j - dO_i . O_i)
+ *   dQ_i = scale * sum_j dS_ij k_j,   dK_j = scale * sum_i dS_ij q_i
+ *
+ * (dO_i . O_i equals sum_j P_ij dO_i . v_j, the row term of the softmax
+ * Jacobian.)
+ *
+ *   q, k, v, o, dout : device, bf16 [B, H, n, d], 16-byte aligned, read only;
+ *                      o and lse are attn_fwd's outputs for q, k, v
+ *   lse              : device, fp32 [B, H, n], 4-byte aligned, read only
+ *   dq, dk, dv       : device, bf16 [B, H, n, d], 16-byte aligned, written
+ *   workspace        : device scratch owned by the caller, 16-byte aligned,
+ *                      at least attn_bwd_workspace_bytes(B, H, n, d) bytes
+ *                      (an fp32 dQ accumulator and two fp32 per-row arrays);
+ *                      its contents on entry do not matter, and it must not
+ *                      be used by other work until this call's work is done
+ *   B, H, n, d, scale, causal, window, stream : as attn_fwd (K and V have H
+ *                      heads: the grouped-query form has no backward here)
+ *
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation; P and dS
+ * are rounded to bf16 before their products; dQ is accumulated in fp32 over
+ * key tiles (atomic adds, so its last bits may differ between runs); dQ, dK,
+ * dV are rounded to bf16 once. Three kernels are enqueued on `stream`.
+ * Returns as attn_fwd; ATTN_ERR_INVALID also for a short or misaligned
+ * workspace. Outputs must not overlap inputs or the workspace.
+ */
+ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                      const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                      void *workspace, size_t workspace_bytes, int B, int H, int n, int d,
+                      float scale, int causal, int window, void *stream);
+
+/* Device workspace bytes attn_bwd needs for this shape, or -1 if the shape
+ * is invalid or unsupported. */
+ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
+
+/*
  * attn_sync_status - synchronize `stream`, then read and clear this device's
  * status word. Returns ATTN_ERR_TIMEOUT if any kernel since the last call gave
  * up on a bounded wait (its outputs are then undefined), ATTN_ERR_CUDA if the
- * synchronization reported a CUDA error, else ATTN_OK.
+ * synchronization reported a CUDA error or a kernel found its shared memory
+ * unusable and did no work, else ATTN_OK.
  */
 ATTN_API int attn_sync_status(void *stream);
 

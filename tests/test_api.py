@@ -130,3 +130,42 @@ def test_binding_checks_grouped_shapes(attn):
         attn._check_qkv(q, kv, kv, device=False, grouped=True)
     kv2 = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
     attn._check_qkv(q, kv2, kv2, device=False, grouped=True)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), 1), (dict(dout=0), 1), (dict(dq=0), 1), (dict(workspace=0), 1), (dict(lse=0), 1),
+    (dict(B=0), 1), (dict(n=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(causal=2), 1), (dict(dk=FAKE + 8), 1), (dict(workspace=FAKE + 4), 1), (dict(lse=FAKE + 2), 1),
+    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(causal=0, window=5), 2), (dict(n=(1 << 30) + 1), 2),
+    (dict(B=1 << 16, H=1 << 16), 1),
+])
+def test_attn_bwd_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+             workspace=FAKE, ws_bytes=1 << 40, B=1, H=1, n=128, d=64, scale=0.125, causal=1,
+             window=-1, stream=None)
+    a.update(kw)
+    rc = attn.lib().attn_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"], a["dk"],
+                             a["dv"], a["workspace"], a["ws_bytes"], a["B"], a["H"], a["n"], a["d"],
+                             a["scale"], a["causal"], a["window"], a["stream"])
+    assert rc == code
+
+
+def test_bwd_workspace_size(attn):
+    # fp32 dQ accumulator + two fp32 per-row arrays padded to 128-row tiles,
+    # each part rounded up to 256 bytes
+    def expect(B, H, n, d):
+        r = lambda x: (x + 255) // 256 * 256
+        n_pad = (n + 127) // 128 * 128
+        return r(B * H * n * d * 4) + 2 * r(B * H * n_pad * 4)
+    for shape in [(1, 1, 1, 64), (1, 2, 300, 64), (2, 3, 129, 128), (8, 8, 8192, 64)]:
+        assert attn.bwd_workspace_bytes(*shape) == expect(*shape)
+    assert attn.lib().attn_bwd_workspace_bytes(1, 1, 128, 80) == -1
+    assert attn.lib().attn_bwd_workspace_bytes(0, 1, 128, 64) == -1
+
+
+def test_bwd_binding_checks_tensors_before_calling(attn):
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 8)
+    with pytest.raises(ValueError):
+        attn.attn_bwd(q, q, q, q, lse, q)  # host tensors

@@ -1,0 +1,124 @@
+"""Backward pass (through the C ABI) against the fp64 backward oracle.
+
+The GPU side runs the product pipeline: attn_fwd gives O and LSE, attn_bwd
+takes them with dO. The oracle computes dQ, dK, dV from Q, K, V and dO
+alone. Small problems are compared in full (several 128-row tiles, ragged
+tails, every mask); full-size workloads are compared on sampled query rows
+(dQ) and sampled key rows of a few heads (dK, dV), plus invariants.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_softmax_attention_04_b200 import synth
+from parity import assert_grads_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def attn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    import exact_softmax_attention_04_b200 as pkg
+    return pkg
+
+
+def _fwd_bwd(attn, q, k, v, do, causal, window, scale=None, workspace=None):
+    qc, kc, vc, doc = (x.cuda() for x in (q, k, v, do))
+    o, lse = attn.attn_fwd(qc, kc, vc, scale, causal, window)
+    dq, dk, dv = attn.attn_bwd(qc, kc, vc, o, lse, doc, scale, causal, window, workspace=workspace)
+    assert attn.sync_status() == attn.ATTN_OK
+    return dq, dk, dv
+
+
+def _np(t):
+    return t.float().cpu().numpy()
+
+
+MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 127), (True, 128), (True, 129),
+         (True, 300), (True, 100000)]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n", [1, 77, 128, 129, 256, 383, 640])
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_bwd_small_shapes_all_masks_in_full(attn, oracle_mod, d, n, causal, window):
+    q_std = 4.0 if (n + d + window) % 2 else 1.0
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=n * 7 + d, q_std=q_std)
+    do = synth.make_dout(1, 2, n, d, seed=n * 7 + d)
+    sc = 1.0 / np.sqrt(d)
+    grads = _fwd_bwd(attn, q, k, v, do, causal, window)
+    refs = oracle_mod.attn_bwd(q, k, v, do, sc, causal, window)
+    assert_grads_close([_np(g) for g in grads], refs, f"n{n} d{d} c{causal} w{window}")
+
+
+def test_bwd_batch_heads_and_scale(attn, oracle_mod):
+    q, k, v = synth.make_qkv(3, 5, 200, 64, seed=60)
+    do = synth.make_dout(3, 5, 200, 64, seed=60)
+    for causal, window, scale in [(False, -1, 0.125), (True, -1, 0.3), (True, 50, 0.05)]:
+        grads = _fwd_bwd(attn, q, k, v, do, causal, window, scale)
+        refs = oracle_mod.attn_bwd(q, k, v, do, scale, causal, window)
+        assert_grads_close([_np(g) for g in grads], refs, f"B3H5 c{causal} w{window} s{scale}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_window_zero(attn, d):
+    """w = 0: P is the identity, so dV = dO exactly and dQ, dK vanish (up to
+    the rounding of dO.v - dO.O, both of which equal dO.v)."""
+    q, k, v = synth.make_qkv(2, 2, 257, d, seed=61, q_std=4.0)
+    do = synth.make_dout(2, 2, 257, d, seed=61)
+    dq, dk, dv = _fwd_bwd(attn, q, k, v, do, True, 0)
+    assert torch.equal(dv.cpu(), do)
+    assert dq.float().abs().max().item() <= 1e-3
+    assert dk.float().abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 200)])
+def test_bwd_softmax_invariants(attn, causal, window):
+    """sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i per head (rows of P sum to 1)."""
+    q, k, v = synth.make_qkv(1, 4, 1000, 128, seed=62, q_std=2.0)
+    do = synth.make_dout(1, 4, 1000, 128, seed=62)
+    dq, dk, dv = _fwd_bwd(attn, q, k, v, do, causal, window)
+    dk64, dv64 = dk.double().cpu(), dv.double().cpu()
+    ksum = dk64.sum(dim=2).abs().max().item()
+    assert ksum <= 2e-2 * dk64.abs().sum(dim=2).max().item() / np.sqrt(1000), ksum
+    vs = dv64.sum(dim=2) - do.double().sum(dim=2)
+    assert vs.abs().max().item() <= 1e-2 * do.double().abs().sum(dim=2).max().item() / np.sqrt(1000)
+
+
+def test_bwd_dk_dv_deterministic_and_dirty_workspace(attn):
+    """dK and dV come from one CTA each (bit-identical across runs); dQ sums
+    key tiles with atomics (equal up to the order of fp32 adds). A workspace
+    full of garbage gives the same result: the prep kernel resets it."""
+    q, k, v = synth.make_qkv(1, 4, 1000, 64, seed=63)
+    do = synth.make_dout(1, 4, 1000, 64, seed=63)
+    ws = torch.full((attn.bwd_workspace_bytes(1, 4, 1000, 64),), 0x7f, dtype=torch.uint8, device="cuda")
+    a = _fwd_bwd(attn, q, k, v, do, True, 300, workspace=ws)
+    b = _fwd_bwd(attn, q, k, v, do, True, 300)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2 * a[0].float().abs().max().item()
+
+
+@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768], ids=lambda w: w.name)
+def test_bwd_full_size_workloads_sampled(attn, oracle_mod, wl):
+    q, k, v = synth.make_inputs(wl)
+    do = synth.make_dout(wl.B, wl.H, wl.n, wl.d, seed=wl.seed)
+    grads = _fwd_bwd(attn, q, k, v, do, wl.causal, wl.window, wl.scale)
+    qrows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=4, bound_every=1024, edge=4)
+    # key rows of two heads (first and last): their columns need every row of
+    # the head's softmax statistics in the oracle
+    rng = np.random.default_rng(5)
+    heads = [0, wl.B * wl.H - 1]
+    krows = np.concatenate([h * wl.n + np.unique(np.concatenate(
+        [rng.integers(0, wl.n, 48), [0, 127, 128, wl.n - 1]])) for h in heads])
+    dq_ref, dk_ref, dv_ref = oracle_mod.attn_bwd_rows(q, k, v, do, wl.scale, wl.causal, wl.window,
+                                                      qrows, krows)
+    d = wl.d
+    sel = lambda t, rows: t.view(-1, d)[torch.as_tensor(rows, device=t.device)].float().cpu().numpy()
+    assert_grads_close([sel(grads[0], qrows), sel(grads[1], krows), sel(grads[2], krows)],
+                       [dq_ref, dk_ref, dv_ref], wl.name)
+    for g in grads:
+        assert bool(torch.isfinite(g.float()).all())
