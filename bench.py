@@ -401,6 +401,120 @@ def run_ours(args, wl, world, rank, local):
     return 0
 
 
+BWD_METRIC = "attention bwd TFLOP/s (10*d FLOPs per attended pair: five matmuls)"
+
+
+def run_bwd(args, wl, world, rank, local):
+    """Backward pass of one workload: O and LSE from attn_fwd (untimed), then
+    attn_bwd timed as one step (its three launches). FLOPs: five matmuls of
+    2*d per attended pair (S, dP, dV, dK, dQ)."""
+    import numpy as np
+    import exact_softmax_attention_04_b200 as attn
+    from exact_softmax_attention_04_b200 import synth
+
+    if wl.kv_heads != wl.H:
+        raise SystemExit("the backward pass takes K and V with H heads")
+    dev = torch.device("cuda", local)
+    q, k, v = synth.make_inputs(wl)
+    do = synth.make_dout(wl.B, wl.H, wl.n, wl.d, seed=wl.seed)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    o, lse = attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, stream=stream)
+    ws = torch.empty(attn.bwd_workspace_bytes(wl.B, wl.H, wl.n, wl.d), dtype=torch.uint8, device=dev)
+    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H
+    flops = 10 * wl.d * pairs
+    grads = None
+
+    def step():
+        nonlocal grads
+        grads = attn.attn_bwd(qd, kd, vd, o, lse, dod, wl.scale, wl.causal, wl.window, workspace=ws,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local if not args.profile else -1) as clocks:
+        if not args.profile:
+            time.sleep(0.5)
+        wall0 = time.time()
+        start_all, end_all = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start_all.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        end_all.record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+    barrier(world)
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    total_ms = max_over_ranks(start_all.elapsed_time(end_all), world)
+    per_step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    achieved = flops / (per_step_ms / 1e3) / 1e12
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": wl.name, "pass": "bwd", "steps": args.steps,
+                              "ms_per_step": per_step_ms, "tflops": achieved}), flush=True)
+        return 0
+    if rank != 0:
+        return 0
+    bf16_peak, _, peak_src = peaks()
+    line = {
+        "metric": BWD_METRIC, "value": world * flops * args.steps / (total_ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**wl.describe(), "pass": "backward", "dout": "N(0,1), seed + 1",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "no flush: inputs Q, K, V, O, dO exceed the 126 MB L2"
+                         if 5 * q.numel() * 2 > 126e6 else "no flush: inputs fit in L2"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": achieved / bf16_peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "algorithmic_flops_per_launch": flops,
+                     "note": "achieved over the whole attn_bwd call (prep, main and dQ conversion "
+                             "kernels)"},
+        "e2e": {"value": None, "unit": "TFLOP/s",
+                "note": "the backward pass has no host-buffer entry point"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(wall0, wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        g = torch.Generator().manual_seed(2)
+        total = wl.B * wl.H * wl.n
+        flops_per_row = flops / total
+        probe = torch.randint(0, total, (16,), generator=g).numpy()
+        t0 = time.perf_counter()
+        oracle.attn_bwd_rows(q, k, v, do, wl.scale, wl.causal, wl.window, probe, [])
+        dt = max(time.perf_counter() - t0, 1e-3)
+        nrows = int(min(total, max(16, 16 * args.cpu_seconds / dt)))
+        rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
+        t0 = time.perf_counter()
+        dq_ref, _, _ = oracle.attn_bwd_rows(q, k, v, do, wl.scale, wl.causal, wl.window, rows, [])
+        dt = time.perf_counter() - t0
+        dq_gpu = grads[0].view(-1, wl.d)[torch.as_tensor(rows, device=dev)].float().cpu().numpy()
+        diff = dq_gpu - dq_ref
+        line["cpu_baseline"] = {
+            "value": nrows * flops_per_row / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"dQ of {nrows} random query rows (seed 2) of {wl.name}, fp64 oracle, counted at "
+                      "the backward's per-row share of FLOPs",
+            "parity_vs_gpu": {"rows": nrows, "dq_rel_rms": float(np.sqrt((diff ** 2).sum() / (dq_ref ** 2).sum())),
+                              "dq_max_abs": float(np.abs(diff).max())}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """Kernel time of every target workload (one line each): TFLOP/s on
     unmasked FLOPs, % of the measured peak and HBM GB/s on the minimum bytes
@@ -457,6 +571,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every target workload (kernel only, median of --steps, L2 flushed)")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (attn_bwd) of --workload instead of the forward")
     ap.add_argument("--profile", action="store_true",
                     help="timed kernel launches only (no e2e, CPU baseline or clock sampling): "
                          "the command profiled under ncu")
@@ -474,6 +590,8 @@ def main():
         return run_reference(args, wl, _env_int("WORLD_SIZE", 1), _env_int("RANK", 0))
     world, rank, local = dist_setup(args.gpus)
     try:
+        if args.bwd:
+            return run_bwd(args, wl, world, rank, local)
         return run_ours(args, wl, world, rank, local)
     finally:
         if world > 1:

@@ -35,6 +35,22 @@ BwdWorkspace workspace_layout(int64_t bh, int64_t n, int64_t d)
     return w;
 }
 
+// The fp32 dQ accumulator [bh, n, d] as a 3-D tensor for TMA reduce-adds:
+// boxes of 32 columns (128 bytes) x 128 rows, 128-byte swizzle; rows past n
+// are skipped.
+bool encode_acc(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, float *ptr, int64_t bh, int64_t n,
+                int64_t d)
+{
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                          static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 4), static_cast<cuuint64_t>(n * d * 4)};
+    cuuint32_t box[3] = {32, static_cast<cuuint32_t>(attn_sm100::BM), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int check_bwd_args(int B, int H, int n, int d, float scale, int causal, int window)
 {
     if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return ATTN_ERR_INVALID;
@@ -61,7 +77,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     auto enc = encoder();
     if (!enc) return ATTN_ERR_CUDA;
     const int64_t bh = static_cast<int64_t>(B) * H;
-    CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
     if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
         !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
         !encode_bhnd(enc, &mdk, dk, bh, n, D) || !encode_bhnd(enc, &mdv, dv, bh, n, D))
@@ -85,6 +101,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     }
     const BwdWorkspace w = workspace_layout(bh, n, D);
     float *acc = reinterpret_cast<float *>(ws);
+    if (!encode_acc(enc, &macc, acc, bh, n, D)) return ATTN_ERR_CUDA;
     float *lse2 = reinterpret_cast<float *>(ws + w.acc_bytes);
     float *delta = reinterpret_cast<float *>(ws + w.acc_bytes + w.stat_bytes);
     const int n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
@@ -113,7 +130,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.window = window < 0 ? -1 : window;
     const unsigned grid = static_cast<unsigned>(bh * p.num_k_tiles);
     attn_sm100::attn_bwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
-                                                                                    mdv, p);
+                                                                                    mdv, macc, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
     // 3. dQ accumulator -> bf16

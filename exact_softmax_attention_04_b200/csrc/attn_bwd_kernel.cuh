@@ -24,8 +24,9 @@
 //        dK  += dS^T Q_i         (dS^T from shared memory, K-major)
 //        dQ_i = dS K_j           (the same dS buffer read MN-major)
 //      dK, dV accumulate in TMEM over the whole walk and are stored once;
-//      each dQ_i tile is added into the fp32 accumulator with vector atomics
-//      (several key tiles contribute to every query row).
+//      each dQ_i tile is added into the fp32 accumulator by TMA bulk
+//      reduce-adds from shared memory (several key tiles contribute to every
+//      query row).
 //   3. attn_bwd_dq_convert_kernel: fp32 dQ accumulator -> bf16 dQ.
 //
 // Roles of the main kernel (512 threads, 16 warps = 4 warpgroups):
@@ -38,7 +39,9 @@
 //   warp 9          TMA producer: K_j, V_j once, then Q_i, dO_i and the rows'
 //                   LSE and delta into a two-stage ring.
 //   warps 10-11     idle.
-//   warps 12-15     dQ drain: TMEM -> registers -> atomic add into fp32.
+//   warps 12-15     dQ drain: TMEM -> registers (times scale) -> swizzled fp32
+//                   staging in shared memory -> TMA reduce-add into the
+//                   accumulator, 64 columns (32 KB) at a time.
 // Registers: launched at 128 per thread; the softmax warpgroups raise to 184,
 // the dQ warpgroup drops to 88 and the MMA/TMA warpgroup to 56
 // (2*184 + 88 + 56 = 4*128).
@@ -52,6 +55,14 @@
 namespace attn_sm100 {
 
 constexpr int BWD_NSTAGE = 2;              // Q_i / dO_i ring stages
+
+// Of every 16 pairs of P entries a softmax thread computes, the first
+// ATTN_BWD_EX2_EMU use the FMA-pipe polynomial for 2^x instead of the MUFU
+// (masked entries are zeroed after the exponential, so the polynomial's
+// range limit does not matter there).
+#ifndef ATTN_BWD_EX2_EMU
+#define ATTN_BWD_EX2_EMU 2
+#endif
 constexpr int STATUS_SMEM_ALIGN = 2;       // device status bit: shared memory base not alignable
 
 struct BwdParams {
@@ -81,10 +92,19 @@ struct BwdCfg {
     static constexpr int DO_OFF = Q_OFF + NST * TILE_BYTES;  // + s * TILE_BYTES
     static constexpr int DS_OFF = DO_OFF + NST * TILE_BYTES;
     static constexpr int STAT_OFF = DS_OFF + DS_BYTES;       // + s * 1024: lse2[128], delta[128]
-    static constexpr int BAR_OFF = STAT_OFF + NST * 1024;
+    // dQ staging for the TMA reduce-add: 64 fp32 columns of the 128 query
+    // rows (32 KB, two 128-byte swizzled boxes of 32 columns). D = 64 has a
+    // buffer of its own; D = 128 has no room left and stages its two halves
+    // in the dS buffer, which is idle from the end of dQ_i's MMA until the
+    // softmax writes dS_{i+1}.
+    static constexpr bool DQ_IN_DS = (D == 128);
+    static constexpr int DQS_HALF_BYTES = BM * 64 * 4;
+    static constexpr int DQS_OWN_OFF = STAT_OFF + NST * 1024;
+    static constexpr int BAR_OFF = DQS_OWN_OFF + (DQ_IN_DS ? 0 : DQS_HALF_BYTES);
+    static constexpr int DQS_OFF = DQ_IN_DS ? DS_OFF : DQS_OWN_OFF;
     // kv_full, q_full[NST], q_empty[NST], s_full, dp_full, p_ready, ds_ready,
-    // dq_full, dq_free, ds_free, kv_done, drain
-    static constexpr int NUM_BARS = 10 + 2 * NST;
+    // dq_full, dq_free, ds_free, kv_done, drain, dqs_free
+    static constexpr int NUM_BARS = 11 + 2 * NST;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_USED = MISC_OFF + 16;
     // Slack for aligning the dynamic shared memory base to 1024 bytes (the
@@ -122,6 +142,19 @@ __device__ __forceinline__ void bulk_load_if(uint32_t leader, uint32_t dst, cons
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "r"(leader)
         : "memory");
 }
+
+// 3-D tiled reduce-add shared -> global (fp32 add in L2; rows outside the
+// tensor are skipped), tracked by the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+                 " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// Wait until every bulk async-group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr)
 {
@@ -217,7 +250,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                    const BwdParams p)
+                    const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p)
 {
     using C = BwdCfg<D>;
     constexpr int NST = C::NST;
@@ -243,7 +276,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const uint32_t s_full = bars + 8u * (1 + 2 * NST);
     const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
     const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, ds_free = s_full + 48;
-    const uint32_t kv_done = s_full + 56, drain_bar = s_full + 64;
+    const uint32_t kv_done = s_full + 56, drain_bar = s_full + 64, dqs_free = s_full + 72;
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
@@ -274,6 +307,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         mbar_init(ds_free, 1);
         mbar_init(kv_done, 1);
         mbar_init(drain_bar, 1);
+        mbar_init(dqs_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -338,46 +372,49 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const uint64_t k_mn = smem_desc_sw128(sK, BOX_BYTES, 1024);
         const uint64_t ds_kmaj = smem_desc_sw128(sDS, 16, 1024);
         const uint64_t ds_mn = smem_desc_sw128(sDS, BOX_BYTES, 1024);
-        for (int it = 0; ok && it < nq; ++it) {
-            const int s = it % NST;
-            if (!__all_sync(0xffffffffu, wt.wait(q_full(s), (it / NST) & 1u))) {
-                ok = false;
-                break;
-            }
+        auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+            if (!__all_sync(0xffffffffu, wt.wait(bar, parity))) return false;
             tc_fence_after();
-            const uint64_t q_kmaj = smem_desc_sw128(sQ(s), 16, 1024);
-            const uint64_t do_kmaj = smem_desc_sw128(sdO(s), 16, 1024);
-            const uint64_t q_mn = smem_desc_sw128(sQ(s), BOX_BYTES, 1024);
-            const uint64_t do_mn = smem_desc_sw128(sdO(s), BOX_BYTES, 1024);
-            // S^T = K Q^T: D/16 MMAs over the head dimension
+            return true;
+        };
+        // S^T(it) = K Q_it^T: D/16 MMAs over the head dimension
+        auto issue_s = [&](int it) {
+            const uint64_t q_kmaj = smem_desc_sw128(sQ(it % NST), 16, 1024);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
                 mma_bf16_ss_if(leader, tmem + C::S_COL, k_kmaj + off, q_kmaj + off, idesc_t, k > 0 ? 1u : 0u);
             }
             mma_commit_if(leader, s_full);
-            if (D == 128 && it > 0) {
-                // dQ_{i-1} shares dP's columns: the drain must have read it
-                if (!__all_sync(0xffffffffu, wt.wait(dq_free, (it - 1) & 1u))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-            }
-            // dP^T = V dO^T
+        };
+        // dP^T(it) = V dO_it^T
+        auto issue_dp = [&](int it) {
+            const uint64_t do_kmaj = smem_desc_sw128(sdO(it % NST), 16, 1024);
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
                 const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
                 mma_bf16_ss_if(leader, tmem + C::DP_COL, v_kmaj + off, do_kmaj + off, idesc_t, k > 0 ? 1u : 0u);
             }
             mma_commit_if(leader, dp_full);
+        };
+        // Issue order: S(0), dP(0), then per query tile it
+        //   dV(it), S(it+1), dK(it), dQ(it), dP(it+1).
+        // S(it+1) overwrites P(it) in TMEM right behind dV(it), its reader
+        // (MMAs complete in issue order), so the softmax warps can start on
+        // tile it+1 as soon as they have produced dS(it), while the tensor
+        // core runs dK(it) and dQ(it).
+        if (ok) ok = wait(q_full(0), 0);
+        if (ok) {
+            issue_s(0);
+            issue_dp(0);
+        }
+        for (int it = 0; ok && it < nq; ++it) {
+            const int s = it % NST;
+            const uint64_t q_mn = smem_desc_sw128(sQ(s), BOX_BYTES, 1024);
+            const uint64_t do_mn = smem_desc_sw128(sdO(s), BOX_BYTES, 1024);
             // dV += P^T dO: 8 MMAs of 16 queries; P^T of queries [0,64) is in
             // TMEM columns [0,32), of queries [64,128) in [64,96)
-            if (!__all_sync(0xffffffffu, wt.wait(p_ready, it & 1u))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+            if (!(ok = wait(p_ready, it & 1u))) break;
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk) {
                 const uint32_t pcol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
@@ -385,18 +422,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                                do_mn + static_cast<uint64_t>(kk * 128), idesc_acc,
                                (it > 0 || kk > 0) ? 1u : 0u);
             }
-            if (!__all_sync(0xffffffffu, wt.wait(ds_ready, it & 1u))) {
-                ok = false;
-                break;
+            if (it + 1 < nq) {
+                if (!(ok = wait(q_full((it + 1) % NST), ((it + 1) / NST) & 1u))) break;
+                issue_s(it + 1);
             }
-            tc_fence_after();
-            if (D == 64 && it > 0) {
-                if (!__all_sync(0xffffffffu, wt.wait(dq_free, (it - 1) & 1u))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-            }
+            if (!(ok = wait(ds_ready, it & 1u))) break;
+            if (D == 64 && it > 0 && !(ok = wait(dq_free, (it - 1) & 1u))) break;
             // dK += dS^T Q: dS^T K-major (keys are rows), Q MN-major
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk) {
@@ -404,7 +435,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 mma_bf16_ss_if(leader, tmem + C::DK_COL, ds_kmaj + off, q_mn + static_cast<uint64_t>(kk * 128),
                                idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
             }
-            // dQ_i = dS K: the same buffer read with queries as rows (MN-major)
+            // dQ_it = dS K: the same buffer read with queries as rows (MN-major)
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
                 mma_bf16_ss_if(leader, tmem + C::DQ_COL, ds_mn + static_cast<uint64_t>(kk * 128),
@@ -412,6 +443,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             mma_commit_if(leader, dq_full);
             mma_commit_if(leader, ds_free);
             mma_commit_if(leader, q_empty(s));
+            if (it + 1 < nq) {
+                // with D = 128, dQ_it sits in dP's columns: the drain must have read it
+                if (D == 128 && !(ok = wait(dq_free, it & 1u))) break;
+                issue_dp(it + 1);
+            }
         }
         if (ok) mma_commit_if(leader, kv_done);
         // Every MMA this warp issued must finish before TMEM is freed.
@@ -422,28 +458,59 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // ------------------------------------------------------------ dQ drain
         regs_decrease<C::REGS_DQ>();
         const int r = threadIdx.x % BM;  // query row in the tile == TMEM lane
+        const bool issuer = (r == 0);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
         const float sc = p.scale;
-        for (int it = 0; it < nq; ++it) {
-            if (!__all_sync(0xffffffffu, wt.wait(dq_full, it & 1u))) break;
-            tc_fence_after();
-            const int q = (qlo + it) * BM + r;
-            float *dst = p.dq_acc + (static_cast<size_t>(bh) * n + q) * D;
-#pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
-                uint32_t v[32];
-                tmem_ld32(lane_base + C::DQ_COL + c, v);
-                if (q < n) {
+        const uint32_t stage = base + C::DQS_OFF;
+        // 32 columns of row r (times scale) into staging box b: 16-byte chunk
+        // j of the 128-byte row lands at chunk j ^ (r % 8), the 128-byte
+        // swizzle the tensor map uses.
+        auto stage32 = [&](const uint32_t (&v)[32], int b) {
+            const uint32_t rowp = stage + b * (BM * 128) + r * 128;
 #pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + c + 4 * g),
-                                  make_float4(u2f(v[4 * g]) * sc, u2f(v[4 * g + 1]) * sc,
-                                              u2f(v[4 * g + 2]) * sc, u2f(v[4 * g + 3]) * sc));
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t chunk = static_cast<uint32_t>(j) ^ static_cast<uint32_t>(r & 7);
+                st_shared_v4(rowp + chunk * 16, f2u(u2f(v[4 * j]) * sc), f2u(u2f(v[4 * j + 1]) * sc),
+                             f2u(u2f(v[4 * j + 2]) * sc), f2u(u2f(v[4 * j + 3]) * sc));
+            }
+        };
+        for (int it = 0; it < nq; ++it) {
+            // all four warps take the same decision (they meet at named
+            // barriers below)
+            if (!named_bar_and(3, BM, wt.wait(dq_full, it & 1u))) break;
+            tc_fence_after();
+            const int q0 = (qlo + it) * BM;
+#pragma unroll 1
+            for (int hf = 0; hf < D / 64; ++hf) {
+                uint32_t va[32], vb[32];
+                tmem_ld32(lane_base + C::DQ_COL + 64 * hf, va);
+                tmem_ld32(lane_base + C::DQ_COL + 64 * hf + 32, vb);
+                if (hf == D / 64 - 1) {
+                    // dQ_i is in registers: its TMEM columns may be reused
+                    tc_fence_before();
+                    mbar_arrive(dq_free);
+                }
+                // the previous reduce-add must have read the staging buffer
+                if (issuer) tma_store_wait_read0();
+                named_bar_sync(3, BM);
+                stage32(va, 0);
+                stage32(vb, 1);
+                fence_proxy_async_smem();
+                named_bar_sync(3, BM);
+                if (issuer) {
+                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, bh);
+                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, bh);
+                    tma_store_commit();
                 }
             }
-            tc_fence_before();
-            mbar_arrive(dq_free);
+            if (C::DQ_IN_DS && issuer) {
+                // the staging used the dS buffer: hand it back to the softmax
+                tma_store_wait_read0();
+                mbar_arrive(dqs_free);
+            }
         }
+        // every reduce-add must be complete before the kernel ends
+        if (issuer) bulk_wait_all();
     } else {
         // ------------------------------------------------------------ softmax / dS
         regs_increase<C::REGS_SOFTMAX>();
@@ -482,7 +549,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                                              make_float2(sc, sc), make_float2(-l4.x, -l4.y));
                     const float2 x23 = ffma2(make_float2(u2f(sv[4 * g + 2]), u2f(sv[4 * g + 3])),
                                              make_float2(sc, sc), make_float2(-l4.z, -l4.w));
-                    float e[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), ex2_approx(x23.y)};
+                    // pairs 16*c2 + 2g and 16*c2 + 2g + 1 of the thread's 32
+                    float e[4];
+                    if ((2 * g) % 16 < ATTN_BWD_EX2_EMU) {
+                        ex2_poly_x2(x01.x, x01.y, e[0], e[1]);
+                    } else {
+                        e[0] = ex2_approx(x01.x);
+                        e[1] = ex2_approx(x01.y);
+                    }
+                    if ((2 * g + 1) % 16 < ATTN_BWD_EX2_EMU) {
+                        ex2_poly_x2(x23.x, x23.y, e[2], e[3]);
+                    } else {
+                        e[2] = ex2_approx(x23.x);
+                        e[3] = ex2_approx(x23.y);
+                    }
                     if (need_mask) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
@@ -505,8 +585,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             ok = __all_sync(0xffffffffu, wt.wait(dp_full, it & 1u));
             if (!ok) break;
             if (it > 0) {
-                // dK_{i-1} and dQ_{i-1} must have read the dS buffer
-                ok = __all_sync(0xffffffffu, wt.wait(ds_free, (it - 1) & 1u));
+                // dK_{i-1} and dQ_{i-1} must have read the dS buffer (and, at
+                // D = 128, the dQ drain must have finished staging in it)
+                ok = __all_sync(0xffffffffu, wt.wait(C::DQ_IN_DS ? dqs_free : ds_free, (it - 1) & 1u));
                 if (!ok) break;
             }
             tc_fence_after();
