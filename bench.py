@@ -525,7 +525,7 @@ def run_sweep(args):
     torch.cuda.set_device(0)
     bf16_peak, hbm_peak, peak_src = peaks()
     wls = [synth.SMALL_CAUSAL, synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072,
-           synth.GQA_N8192] + synth.sweep()
+           synth.GQA_N8192, synth.SYM_N16384] + synth.sweep()
     for wl in wls:
         q, k, v = synth.make_inputs(wl)
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()

@@ -134,7 +134,8 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     q: bf16 CUDA tensor [B, H, n, d]; k, v: [B, H, n, d], or [B, Hkv, n, d]
     with Hkv dividing H for grouped-query / multi-query attention (query
     head h reads key/value head h // (H // Hkv)). Contiguous, d in {64, 128}.
-    causal / window: see include/attn.h (window >= 0 needs causal).
+    causal / window: see include/attn.h (window >= 0 without causal is the
+    symmetric window i - window .. i + window).
     Returns (o bf16 [B, H, n, d], lse fp32 [B, H, n]); enqueued on ``stream``
     (default: the current stream), asynchronous like any CUDA op.
     """

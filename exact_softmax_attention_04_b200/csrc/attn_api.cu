@@ -68,6 +68,11 @@ bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const vo
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int effective_window(int n, int window)
+{
+    return (window < 0 || window >= n - 1) ? -1 : window;
+}
+
 int current_device(int *dev)
 {
     if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return ATTN_ERR_CUDA;
@@ -104,7 +109,6 @@ int check_args(const void *q, const void *k, const void *v, const void *o, const
                            !aligned(o, 16) || !aligned(lse, 4)))
         return ATTN_ERR_INVALID;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (window >= 0 && !causal) return ATTN_ERR_UNSUPPORTED;
     if (n > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
     const int64_t tiles = bh * ((n + attn_sm100::BM - 1) / attn_sm100::BM);
     if (tiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
@@ -155,7 +159,7 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.num_cta_tiles = (p.num_q_tiles + attn_sm100::QT - 1) / attn_sm100::QT;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
-    p.window = window < 0 ? -1 : window;
+    p.window = effective_window(n, window);
     const unsigned grid = static_cast<unsigned>(bh * p.num_cta_tiles);
     attn_sm100::attn_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -280,7 +284,7 @@ extern "C" const char *attn_strerror(int status)
     switch (status) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_INVALID: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head size must be 64 or 128; a window needs causal=1)";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head size must be 64 or 128, n at most 2^30)";
     case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
     case ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait; outputs are undefined";
     case ATTN_ERR_TOO_LARGE: return "problem larger than the fixed scratch of attn_fwd_host_noalloc";
@@ -290,7 +294,12 @@ extern "C" const char *attn_strerror(int status)
 
 extern "C" int64_t attn_attended_pairs(int64_t n, int causal, int64_t window)
 {
-    if (n < 0 || (window >= 0 && !causal)) return -1;
+    if (n < 0) return -1;
+    if (window >= 0 && !causal) {
+        // symmetric window: sum_i min(n-1, i+w) - max(0, i-w) + 1
+        if (window >= n - 1) return n * n;
+        return n * (2 * window + 1) - window * (window + 1);
+    }
     if (window >= 0 && window < n - 1)
         return (window + 1) * (window + 2) / 2 + (n - window - 1) * (window + 1);
     if (causal) return n * (n + 1) / 2;

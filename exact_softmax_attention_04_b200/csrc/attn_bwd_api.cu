@@ -61,7 +61,6 @@ int check_bwd_args(int B, int H, int n, int d, float scale, int causal, int wind
     // the fp32 accumulator (4 bytes per element) must be addressable
     if (bh * n > INT64_MAX / (4 * static_cast<int64_t>(d) + 16)) return ATTN_ERR_INVALID;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (window >= 0 && !causal) return ATTN_ERR_UNSUPPORTED;
     if (n > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
     const int64_t ktiles = bh * ((n + attn_sm100::BN - 1) / attn_sm100::BN);
     if (ktiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
@@ -127,7 +126,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
-    p.window = window < 0 ? -1 : window;
+    p.window = effective_window(n, window);
     const unsigned grid = static_cast<unsigned>(bh * p.num_k_tiles);
     attn_sm100::attn_bwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
                                                                                     mdv, macc, p);

@@ -230,12 +230,13 @@ __global__ void __launch_bounds__(256)
 
 // Query tiles [qlo, qhi) holding a query that attends to some key of the key
 // tile starting at k0 (k0 < n): causal queries start at the key tile's own
-// tile; a window ends them at k0 + 127 + window.
+// tile, a symmetric window starts them at k0 - window; any window ends them
+// at k0 + 127 + window.
 __device__ __forceinline__ void query_tile_range(int k0, int n, int causal, int window, int &qlo,
                                                  int &qhi)
 {
     const int nqt = (n + BM - 1) / BM;
-    qlo = causal ? k0 / BM : 0;
+    qlo = causal ? k0 / BM : (window >= 0 ? max(0, k0 - window) / BM : 0);
     qhi = nqt;
     if (window >= 0) {
         const int64_t last = min(static_cast<int64_t>(n) - 1, static_cast<int64_t>(k0) + BN - 1 + window);
@@ -344,6 +345,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             if (it >= NST && !__all_sync(0xffffffffu, wt.wait(q_empty(s), ((it / NST) & 1u) ^ 1u)))
                 break;
             const int q0 = (qlo + it) * BM;
+#ifdef ATTN_FAULT_BWD_DROP_FIRST_Q
+            // Test hook (never defined in the library build): the first Q/dO
+            // stage is never loaded, so the MMA warp's wait on it must expire
+            // and the kernel must stop cleanly.
+            if (it == 0) {
+                ++issued;
+                continue;
+            }
+#endif
             mbar_arrive_expect_tx_if(leader, q_full(s), 2 * C::TILE_BYTES + 1024);
 #pragma unroll
             for (int b = 0; b < C::BOXES; ++b) {
@@ -529,8 +539,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             tc_fence_after();
             // Allowed query columns of this key row: one interval [lo, hi].
             const bool need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
-                                   (window >= 0 && q0 + BM - 1 > k0 + window);
-            int lo = causal ? key - q0 : 0;
+                                   (window >= 0 && q0 + BM - 1 > k0 + window) ||
+                                   (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
+            int lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
             int hi = min(BM - 1, n - 1 - q0);
             if (window >= 0) hi = min(hi, key + window - q0);
             if (key >= n) hi = -1;

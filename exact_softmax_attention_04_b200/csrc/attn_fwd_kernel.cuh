@@ -157,7 +157,9 @@ struct Waiter {
 
 // Key tiles [jlo, jhi) holding at least one key allowed for some row of the
 // query tile starting at m0 (fully masked tiles are never visited). Empty when
-// the query tile lies past n.
+// the query tile lies past n. A window (window >= 0, at most n - 2: the host
+// turns wider windows into no window) limits keys to i - window and, when
+// not causal, to i + window.
 __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int window, int &jlo,
                                                int &jhi)
 {
@@ -165,7 +167,11 @@ __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int wi
         jlo = jhi = 0;
         return;
     }
-    const int kend = causal ? min(n, m0 + BM) : n;  // exclusive
+    int kend = n;  // exclusive
+    if (causal)
+        kend = min(n, m0 + BM);
+    else if (window >= 0)
+        kend = min(n, m0 + BM + window);
     const int kbeg = (window >= 0) ? max(0, m0 - window) : 0;
     jlo = kbeg / BN;
     jhi = (kend + BN - 1) / BN;
@@ -454,11 +460,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
             const int k0 = j * BN;
             const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
-                                   (window >= 0 && k0 < q0 + BM - 1 - window);
+                                   (window >= 0 && k0 < q0 + BM - 1 - window) ||
+                                   (!causal && window >= 0 && k0 + BN - 1 > q0 + window);
             if (need_mask) {
                 // Allowed keys of this row form one interval; in tile columns:
                 // [lo, hi] with key = k0 + column.
-                const int hi = min(causal ? row - k0 : BN - 1, n - 1 - k0);
+                const int hi = min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
+                                   n - 1 - k0);
                 const int lo = (window >= 0) ? row - window - k0 : 0;
 #pragma unroll
                 for (int c = 0; c < BN; ++c)

@@ -31,6 +31,11 @@ int *status_word(int dev);
 bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int64_t bh,
                  int64_t n, int64_t d);
 
+// The window the kernels see: -1 (none) for window < 0 and for windows that
+// reach every key (window >= n - 1, where the mask is the same without it),
+// so kernel index arithmetic never meets a window wider than n.
+int effective_window(int n, int window);
+
 // The calling thread's current device, checked against kMaxDevices.
 int current_device(int *dev);
 

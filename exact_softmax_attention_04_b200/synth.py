@@ -48,7 +48,7 @@ class Workload:
     @property
     def mask(self) -> str:
         if self.window >= 0:
-            return f"window{self.window}"
+            return f"window{self.window}" if self.causal else f"symwindow{self.window}"
         return "causal" if self.causal else "none"
 
     def describe(self) -> dict:
@@ -70,8 +70,15 @@ def attended_pairs_per_head(n: int, causal: bool, window: int) -> int:
     """Number of (query, key) pairs a mask allows in one head.
 
     none: n*n; causal: n(n+1)/2; causal window w: sum over i of
-    min(i, w) + 1. Used only to count the unmasked FLOPs (4*d per pair).
+    min(i, w) + 1; symmetric window w (not causal): sum over i of
+    min(n-1, i+w) - max(0, i-w) + 1 = n(2w+1) - w(w+1) for w < n. Used only
+    to count the unmasked FLOPs (4*d per pair).
     """
+    if window >= 0 and not causal:
+        w = window
+        if w >= n - 1:
+            return n * n
+        return n * (2 * w + 1) - w * (w + 1)
     if window >= 0:
         w = window
         if w >= n - 1:
@@ -146,6 +153,9 @@ CAUSAL_N131072 = Workload("B1-H8-n131072-d128-causal", 1, 8, 131072, 128, True)
 # Grouped-query attention with the head layout the pages quote for LLaMA-2 70B
 # (64 query heads sharing 8 key/value heads), causal, 8192 tokens.
 GQA_N8192 = Workload("B1-H64-Hkv8-n8192-d128-causal", 1, 64, 8192, 128, True, Hkv=8)
+# Symmetric local window (each token sees 256 neighbours on either side, the
+# 512-token span of Longformer-style local attention), d = 64, 16k tokens.
+SYM_N16384 = Workload("B2-H16-n16384-d64-symwindow256", 2, 16, 16384, 64, False, 256)
 
 
 def sweep() -> List[Workload]:
@@ -162,7 +172,7 @@ def sweep() -> List[Workload]:
 
 
 def by_name(name: str) -> Optional[Workload]:
-    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072, GQA_N8192] + sweep():
+    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072, GQA_N8192, SYM_N16384] + sweep():
         if wl.name == name:
             return wl
     return None

@@ -24,8 +24,11 @@
  *                              window; the window-mask snippet on "week17
  *                              efficiency attention", local attention section;
  *                              min(i, window) + 1 keys including i itself)
- *   causal = 0, window >= 0 : ATTN_ERR_UNSUPPORTED (the symmetric window
- *                              i-w .. i+w of the same page is not provided)
+ *   causal = 0, window >= 0 : max(0, i - window) <= j <= min(n - 1, i + window)
+ *                              (symmetric local window: each token attends to
+ *                              its window nearest neighbours on either side;
+ *                              local attention section of the same page)
+ * A window of n - 1 or more allows the same keys as no window.
  *
  * Layout: Q, K, V and O are bf16, contiguous [B, H, n, d] (token-major inside
  * each head, d fastest). LSE is fp32, contiguous [B, H, n], natural-log units.

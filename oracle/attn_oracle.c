@@ -20,6 +20,10 @@
  *            "Efficient Transformers ...", section "Family 3")
  *   window : max(0, i - w) <= j <= i  (the causal sliding-window mask code on
  *            "week17 efficiency attention", section on local attention)
+ *   symmetric window (causal = 0, w >= 0) :
+ *            max(0, i - w) <= j <= min(n - 1, i + w)  (the same page's local
+ *            attention: each token attends to its w nearest neighbours on
+ *            either side)
  * Then, all in fp64 over the bf16-decoded inputs,
  *   s_ij  = scale * sum_c q_ic k_jc          for j in A(i)
  *   M_i   = max_{j in A(i)} s_ij
@@ -95,19 +99,25 @@ int oracle_matmul_f64(int64_t m, int64_t n, int64_t k, const double *A, int ta,
     return 0;
 }
 
+/* Is key j in A(i)? The one definition of the masks (see the top of the file). */
+static int allowed_pair(int64_t i, int64_t j, int causal, int64_t window)
+{
+    if (causal && j > i)
+        return 0;
+    if (window >= 0 && j < i - window)
+        return 0;
+    if (!causal && window >= 0 && j > i + window)
+        return 0;
+    return 1;
+}
+
 /* Explicit mask row: allowed[j] = 1 iff key j is in A(i). */
 int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned char *allowed)
 {
     if (n < 0 || i < 0 || i >= n || !allowed)
         return 1;
-    for (int64_t j = 0; j < n; ++j) {
-        int ok = 1;
-        if (causal && j > i)
-            ok = 0;
-        if (window >= 0 && j < i - window)
-            ok = 0;
-        allowed[j] = (unsigned char)ok;
-    }
+    for (int64_t j = 0; j < n; ++j)
+        allowed[j] = (unsigned char)allowed_pair(i, j, causal, window);
     return 0;
 }
 
@@ -120,7 +130,7 @@ int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned c
  *   lse     : nrows       fp64 output (may be NULL)
  *   weights : nrows x n   fp64 normalised weights, 0 where masked (may be NULL)
  *   kernel  : ORACLE_KERNEL_SOFTMAX or ORACLE_KERNEL_IDENTITY
- * window >= 0 requires causal. Returns 0 on success, nonzero on bad input.
+ * Returns 0 on success, nonzero on bad input.
  */
 int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                              int64_t B, int64_t H, int64_t Hkv, int64_t n, int64_t d,
@@ -131,8 +141,6 @@ int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_
     if (!q || !k || !v || !o || (!rows && nrows) || B <= 0 || H <= 0 || n <= 0 || d <= 0)
         return 1;
     if (Hkv <= 0 || H % Hkv != 0)
-        return 1;
-    if (window >= 0 && !causal)
         return 1;
     if (kernel != ORACLE_KERNEL_SOFTMAX && kernel != ORACLE_KERNEL_IDENTITY)
         return 1;
@@ -359,7 +367,7 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
  *   qrows (nq)    : flat query rows (b*H + h)*n + i whose dQ is wanted -> dq (nq x d)
  *   krows (nk)    : flat key rows (b*H + h)*n + j whose dK, dV are wanted
  *                   -> dk, dv (nk x d each)
- * window >= 0 requires causal. Returns 0 on success, nonzero on bad input.
+ * Returns 0 on success, nonzero on bad input.
  */
 int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const void *dout, int type,
                              int64_t B, int64_t H, int64_t n, int64_t d, double scale, int causal,
@@ -369,8 +377,6 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
     if (!q || !k || !v || !dout || B <= 0 || H <= 0 || n <= 0 || d <= 0)
         return 1;
     if (type != ORACLE_IN_BF16 && type != ORACLE_IN_F64)
-        return 1;
-    if (window >= 0 && !causal)
         return 1;
     if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv)) || nq < 0 || nk < 0)
         return 1;
@@ -443,10 +449,7 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
                 for (int64_t c = 0; c < d; ++c)
                     gk[c] = gv[c] = 0.0;
                 for (int64_t i = 0; i < n; ++i) {
-                    /* is key j in A(i)? */
-                    if (causal && j > i)
-                        continue;
-                    if (window >= 0 && j < i - window)
+                    if (!allowed_pair(i, j, causal, window))
                         continue;
                     double sij = 0.0, dpij = 0.0;
                     for (int64_t c = 0; c < d; ++c) {

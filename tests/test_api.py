@@ -63,10 +63,10 @@ def test_attended_pairs_matches_the_workload_counts(attn):
     from exact_softmax_attention_04_b200 import synth
     for n in (1, 2, 127, 128, 129, 1000, 131072):
         for causal, window in [(False, -1), (True, -1), (True, 0), (True, 1), (True, 256), (True, 4096),
-                               (True, 10 ** 6)]:
+                               (True, 10 ** 6), (False, 0), (False, 1), (False, 256), (False, 10 ** 6)]:
             assert attn.attended_pairs(n, causal, window) == synth.attended_pairs_per_head(n, causal, window)
     with pytest.raises(ValueError):
-        attn.attended_pairs(10, False, 3)
+        attn.attended_pairs(-1, False, 3)
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails validation first
@@ -76,7 +76,7 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case below fails va
     (dict(q=0), 1), (dict(lse=0), 1), (dict(B=0), 1), (dict(H=-1), 1), (dict(n=0), 1),
     (dict(d=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(scale=-1.0), 1),
     (dict(scale=float("inf")), 1), (dict(causal=2), 1), (dict(q=FAKE + 8), 1), (dict(lse=FAKE + 2), 1),
-    (dict(d=96), 2), (dict(d=256), 2), (dict(causal=0, window=5), 2), (dict(n=(1 << 30) + 1), 2),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(n=(1 << 30) + 1), 2),
     (dict(B=1 << 16, H=1 << 16), 1),
 ])
 def test_attn_fwd_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
@@ -136,7 +136,7 @@ def test_binding_checks_grouped_shapes(attn):
     (dict(q=0), 1), (dict(dout=0), 1), (dict(dq=0), 1), (dict(workspace=0), 1), (dict(lse=0), 1),
     (dict(B=0), 1), (dict(n=0), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
     (dict(causal=2), 1), (dict(dk=FAKE + 8), 1), (dict(workspace=FAKE + 4), 1), (dict(lse=FAKE + 2), 1),
-    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(causal=0, window=5), 2), (dict(n=(1 << 30) + 1), 2),
+    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(n=(1 << 30) + 1), 2),
     (dict(B=1 << 16, H=1 << 16), 1),
 ])
 def test_attn_bwd_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):

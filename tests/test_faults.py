@@ -47,3 +47,39 @@ def test_expired_wait_reports_timeout_and_context_survives(tmp_path, oracle_mod)
     assert pkg.sync_status() == pkg.ATTN_OK
     o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, 0.125, False, -1)
     assert_close(o2.float().cpu().numpy(), lse2.cpu().numpy(), o_ref, lse_ref, "after timeout")
+
+
+def test_backward_expired_wait_reports_timeout_and_context_survives(tmp_path, oracle_mod):
+    """The backward kernel's first Q/dO stage is never loaded (test-only
+    ATTN_FAULT_BWD_DROP_FIRST_Q hook): its MMA warp's wait must expire, the
+    call must report ATTN_ERR_TIMEOUT, and the context must stay usable."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import exact_softmax_attention_04_b200 as pkg
+    from exact_softmax_attention_04_b200 import build_lib
+    from parity import assert_grads_close
+    build_lib.build()
+    fault_lib = pkg.load_library(build_lib.build_variant(tmp_path / "libattn_fault_bwd.so",
+                                                         ["ATTN_FAULT_BWD_DROP_FIRST_Q"]))
+    n, d = 384, 64
+    q, k, v = synth.make_qkv(1, 1, n, d, seed=51)
+    do = synth.make_dout(1, 1, n, d, seed=51)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = pkg.attn_fwd(qd, kd, vd, 0.125, True, -1)
+    assert pkg.sync_status() == pkg.ATTN_OK
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    ws = torch.empty(pkg.bwd_workspace_bytes(1, 1, n, d), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.time()
+    rc = fault_lib.attn_bwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            dod.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                            ws.numel(), 1, 1, n, d, 0.125, 1, -1, stream)
+    assert rc == pkg.ATTN_OK
+    st = fault_lib.attn_sync_status(stream)
+    assert st == pkg.ATTN_ERR_TIMEOUT, pkg.strerror(st)
+    assert time.time() - t0 < 30.0
+    assert fault_lib.attn_sync_status(stream) == pkg.ATTN_OK
+    grads = pkg.attn_bwd(qd, kd, vd, o, lse, dod, 0.125, True, -1)
+    assert pkg.sync_status() == pkg.ATTN_OK
+    refs = oracle_mod.attn_bwd(q, k, v, do, 0.125, True, -1)
+    assert_grads_close([g.float().cpu().numpy() for g in grads], refs, "after backward timeout")

@@ -23,8 +23,9 @@ def _brute(q, k, v, scale, causal, window):
     """Textbook masked softmax attention over the full score matrix.
 
     Built the way the pages build it: the full S = Q K^T / sqrt(d), a boolean
-    mask made like the sliding-window snippet (ones on [max(0, i-w), i]) or the
-    triu(1) causal mask, masked_fill with -inf, row softmax, then times V.
+    mask made like the sliding-window snippet (ones on [max(0, i-w), i]), the
+    local-attention range max(0, i-w) ... min(n-1, i+w) when not causal, or
+    the triu(1) causal mask, masked_fill with -inf, row softmax, then times V.
     """
     Q, K, V = _f64(q), _f64(k), _f64(v)
     n = Q.shape[-2]
@@ -32,7 +33,8 @@ def _brute(q, k, v, scale, causal, window):
     if window >= 0:
         keep = np.zeros((n, n), dtype=bool)
         for i in range(n):
-            keep[i, max(0, i - window): i + 1] = True
+            last = i if causal else min(n - 1, i + window)
+            keep[i, max(0, i - window): last + 1] = True
     elif causal:
         keep = ~np.triu(np.ones((n, n), dtype=bool), 1)
     else:
@@ -45,7 +47,8 @@ def _brute(q, k, v, scale, causal, window):
     return P @ V, (M + np.log(Z))[..., 0], P
 
 
-MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 3), (True, 64)]
+MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 3), (True, 64),
+         (False, 0), (False, 1), (False, 3), (False, 64)]
 
 
 @pytest.mark.parametrize("n", [1, 7, 33, 64])
@@ -268,8 +271,6 @@ def test_row_subset_equals_full_run(oracle_mod):
 def test_oracle_rejects_bad_arguments(oracle_mod):
     q, k, v = synth.make_qkv(1, 1, 8, 16)
     with pytest.raises(ValueError):
-        oracle_mod.attn_fwd(q, k, v, 0.25, False, 3)  # window needs causal
-    with pytest.raises(ValueError):
         oracle_mod.attn_rows(q, k, v, 0.25, True, -1, [8])  # row out of range
     _, k2, v2 = synth.make_qkv(1, 1, 8, 16, Hkv=1)
     q2, _, _ = synth.make_qkv(1, 2, 8, 16)
@@ -279,7 +280,8 @@ def test_oracle_rejects_bad_arguments(oracle_mod):
 
 def test_pair_count_matches_explicit_masks(oracle_mod):
     for n in (1, 2, 9, 130):
-        for causal, window in [(False, -1), (True, -1), (True, 0), (True, 3), (True, 128), (True, 500)]:
+        for causal, window in [(False, -1), (True, -1), (True, 0), (True, 3), (True, 128), (True, 500),
+                               (False, 0), (False, 3), (False, 128), (False, 500)]:
             cnt = sum(int(oracle_mod.mask_row(n, i, causal, window).sum()) for i in range(n))
             assert cnt == synth.attended_pairs_per_head(n, causal, window)
 
@@ -330,3 +332,44 @@ def test_gqa_rejects_non_dividing_heads(oracle_mod):
     _, k, v = synth.make_qkv(1, 3, 8, 16)
     with pytest.raises(ValueError):
         oracle_mod.attn_rows_gqa(q, k, v, 0.25, False, -1, [0])
+
+
+# ---------------------------------------------------------------- symmetric window
+
+def test_symmetric_window_matches_page_range(oracle_mod):
+    """Local attention: token i attends to max(0, i-w) ... min(n-1, i+w)."""
+    n = 50
+    for w in (0, 1, 7, 49, 60):
+        for i in range(n):
+            m = oracle_mod.mask_row(n, i, False, w)
+            assert np.flatnonzero(m).tolist() == list(range(max(0, i - w), min(n - 1, i + w) + 1))
+
+
+def test_symmetric_window_at_least_n_minus_1_equals_no_mask(oracle_mod):
+    q, k, v = synth.make_qkv(1, 2, 40, 16, seed=80, q_std=3.0)
+    a = oracle_mod.attn_fwd(q, k, v, 0.25, False, -1)
+    for w in (39, 100):
+        b = oracle_mod.attn_fwd(q, k, v, 0.25, False, w)
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_symmetric_window_zero_and_zero_queries(oracle_mod):
+    q, k, v = synth.make_qkv(1, 2, 30, 16, seed=81, q_std=4.0)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.25, False, 0)
+    np.testing.assert_array_equal(o, _f64(v))
+    z = torch.zeros_like(q)
+    o, lse = oracle_mod.attn_fwd(z, k, v, 0.25, False, 4)
+    V = _f64(v)
+    for i in range(30):
+        lo, hi = max(0, i - 4), min(29, i + 4)
+        np.testing.assert_allclose(o[:, :, i], V[:, :, lo:hi + 1].mean(axis=2), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, i], np.log(hi - lo + 1), rtol=0, atol=1e-12)
+
+
+def test_symmetric_pair_count_closed_form():
+    """sum_i (min(n-1, i+w) - max(0, i-w) + 1) = n(2w+1) - w(w+1) for w < n."""
+    for n in (1, 2, 5, 130, 1000):
+        for w in (0, 1, 3, n - 1, n, 5 * n):
+            direct = sum(min(n - 1, i + w) - max(0, i - w) + 1 for i in range(n))
+            assert synth.attended_pairs_per_head(n, False, w) == direct

@@ -12,7 +12,8 @@ import torch
 
 from exact_softmax_attention_04_b200 import synth
 
-MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 3), (True, 64)]
+MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 3), (True, 64),
+         (False, 0), (False, 2), (False, 64)]
 
 
 def _textbook_forward(q, k, v, scale, causal, window):
@@ -28,6 +29,8 @@ def _textbook_forward(q, k, v, scale, causal, window):
         drop |= j > i
     if window >= 0:
         drop |= j < i - window
+        if not causal:
+            drop |= j > i + window
     return s.masked_fill(drop, float("-inf")).softmax(-1) @ v
 
 
@@ -56,7 +59,7 @@ def test_bwd_matches_central_finite_differences(oracle_mod):
     K and V under each mask."""
     rng = np.random.default_rng(7)
     n, d, scale = 9, 4, 0.6
-    for causal, window in ((False, -1), (True, -1), (True, 2)):
+    for causal, window in ((False, -1), (True, -1), (True, 2), (False, 2)):
         q, k, v, do = (_rand((1, 1, n, d), s) for s in (11, 12, 13, 14))
         dq, dk, dv = oracle_mod.attn_bwd(q, k, v, do, scale, causal, window)
 
@@ -154,8 +157,6 @@ def test_bwd_row_subsets_equal_full_run(oracle_mod):
 def test_bwd_oracle_rejects_bad_arguments(oracle_mod):
     q, k, v = synth.make_qkv(1, 1, 8, 8, seed=53)
     do = q.clone()
-    with pytest.raises(ValueError):
-        oracle_mod.attn_bwd_rows(q, k, v, do, 0.3, False, 3, [0], [0])  # window without causal
     with pytest.raises(ValueError):
         oracle_mod.attn_bwd_rows(q, k, v, do, 0.3, True, -1, [8], [])   # row out of range
     with pytest.raises(ValueError):

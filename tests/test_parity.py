@@ -56,7 +56,7 @@ def test_small_causal_workload_in_full(attn, oracle_mod):
 
 
 MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 127), (True, 128), (True, 129),
-         (True, 300), (True, 100000)]
+         (True, 300), (True, 100000), (False, 0), (False, 1), (False, 127), (False, 200), (False, 100000)]
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -137,8 +137,8 @@ def test_sweep_cells_sampled(attn, oracle_mod, wl):
     _sampled_check(attn, oracle_mod, wl, rows)
 
 
-@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072],
-                         ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072,
+                                synth.SYM_N16384], ids=lambda w: w.name)
 def test_full_size_workloads_sampled(attn, oracle_mod, wl):
     per_head = 16 if wl.n >= 65536 else 24
     rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=per_head, bound_every=64, edge=32)
@@ -188,3 +188,20 @@ def test_gqa_workload_sampled(attn, oracle_mod):
     l_s = lse.view(-1)[idx].cpu().numpy()
     o_ref, lse_ref = oracle_mod.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, rows)
     assert_close(o_s, l_s, o_ref, lse_ref, wl.name)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_symmetric_window_closed_forms(attn, d):
+    """Symmetric window: w = 0 returns V exactly; zero queries give the mean of
+    the values in [max(0, i-w), min(n-1, i+w)] with LSE = ln(count)."""
+    n, w = 333, 40
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=90, q_std=4.0)
+    o, _ = _gpu(attn, q, k, v, False, 0)
+    assert torch.equal(o.cpu(), v)
+    z = torch.zeros_like(q)
+    o, lse = _gpu(attn, z, k, v, False, w)
+    o, lse, vf = o.double().cpu(), lse.double().cpu(), v.double()
+    for i in (0, 1, 39, 40, 41, 127, 128, 200, 292, 293, n - 1):
+        lo, hi = max(0, i - w), min(n - 1, i + w)
+        assert (o[..., i, :] - vf[..., lo:hi + 1, :].mean(dim=-2)).abs().max() <= 2e-2
+        assert (lse[..., i] - np.log(hi - lo + 1)).abs().max() <= 1e-3

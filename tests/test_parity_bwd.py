@@ -39,7 +39,7 @@ def _np(t):
 
 
 MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 127), (True, 128), (True, 129),
-         (True, 300), (True, 100000)]
+         (True, 300), (True, 100000), (False, 0), (False, 1), (False, 127), (False, 200)]
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -76,7 +76,7 @@ def test_bwd_window_zero(attn, d):
     assert dk.float().abs().max().item() <= 1e-3
 
 
-@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 200)])
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 200), (False, 150)])
 def test_bwd_softmax_invariants(attn, causal, window):
     """sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i per head (rows of P sum to 1)."""
     q, k, v = synth.make_qkv(1, 4, 1000, 128, seed=62, q_std=2.0)
@@ -102,7 +102,8 @@ def test_bwd_dk_dv_deterministic_and_dirty_workspace(attn):
     assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2 * a[0].float().abs().max().item()
 
 
-@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.SYM_N16384],
+                         ids=lambda w: w.name)
 def test_bwd_full_size_workloads_sampled(attn, oracle_mod, wl):
     q, k, v = synth.make_inputs(wl)
     do = synth.make_dout(wl.B, wl.H, wl.n, wl.d, seed=wl.seed)
