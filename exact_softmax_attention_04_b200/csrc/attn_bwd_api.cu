@@ -1,5 +1,6 @@
 // attn_bwd_api.cu - host side of the backward pass: argument checks, workspace
-// layout, TMA descriptors and the three launches. Contracts in include/attn.h.
+// layout, TMA descriptors and the three launches (prep, dK/dV, dQ).
+// Contracts in include/attn.h.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -8,6 +9,7 @@
 #include <cstdint>
 
 #include "attn.h"
+#include "attn_bwd_fused_kernel.cuh"
 #include "attn_bwd_kernel.cuh"
 #include "attn_host.h"
 
@@ -19,8 +21,14 @@ bool g_bwd_set[kMaxDevices][2] = {};
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace layout: [dQ accumulator fp32 B*H*n*d | lse2 fp32 B*H*n_pad |
-// delta fp32 B*H*n_pad], each part starting on a 256-byte boundary.
+// Head size 64 runs the fused kernel (dQ by reduce-adds into an fp32
+// accumulator), head size 128 the split dK/dV and dQ kernels: each is the
+// faster of the two designs measured at that head size.
+bool fused_for(int d) { return d == 64; }
+
+// Workspace layout: [dQ accumulator fp32 B*H*n*d (fused path only) |
+// lse2 fp32 B*H*n_pad | delta fp32 B*H*n_pad], each part starting on a
+// 256-byte boundary (n_pad = n rounded up to 128).
 struct BwdWorkspace {
     size_t acc_bytes, stat_bytes, total;
 };
@@ -29,7 +37,7 @@ BwdWorkspace workspace_layout(int64_t bh, int64_t n, int64_t d)
 {
     const int64_t n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
     BwdWorkspace w;
-    w.acc_bytes = round256(static_cast<size_t>(bh * n * d) * 4);
+    w.acc_bytes = fused_for(static_cast<int>(d)) ? round256(static_cast<size_t>(bh * n * d) * 4) : 0;
     w.stat_bytes = round256(static_cast<size_t>(bh * n_pad) * 4);
     w.total = w.acc_bytes + 2 * w.stat_bytes;
     return w;
@@ -51,7 +59,7 @@ bool encode_acc(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, float *pt
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int check_bwd_args(int B, int H, int n, int d, float scale, int causal, int window)
+int check_bwd_args(int B, int H, int n, int d, float scale, int causal)
 {
     if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return ATTN_ERR_INVALID;
     if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
@@ -62,8 +70,22 @@ int check_bwd_args(int B, int H, int n, int d, float scale, int causal, int wind
     if (bh * n > INT64_MAX / (4 * static_cast<int64_t>(d) + 16)) return ATTN_ERR_INVALID;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (n > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
-    const int64_t ktiles = bh * ((n + attn_sm100::BN - 1) / attn_sm100::BN);
-    if (ktiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    const int64_t tiles = bh * ((n + attn_sm100::BN - 1) / attn_sm100::BN);
+    if (tiles > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// The register split between warpgroups needs exactly the per-thread count it
+// was computed for; refuse a build that differs (its raising warps would wait
+// forever), and allow the kernel its dynamic shared memory.
+template <typename Kernel>
+int prepare_kernel(Kernel kernel, int smem_bytes, uint32_t regs_launch)
+{
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (fa.numRegs != static_cast<int>(regs_launch)) return ATTN_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
     return ATTN_OK;
 }
 
@@ -72,7 +94,74 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
                const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int n,
                float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
 {
-    using Cfg = attn_sm100::BwdCfg<D>;
+    using KV = attn_sm100::BwdKVCfg<D>;
+    using QC = attn_sm100::BwdQCfg<D>;
+    auto enc = encoder();
+    if (!enc) return ATTN_ERR_CUDA;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
+        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
+        !encode_bhnd(enc, &mdq, dq, bh, n, D) || !encode_bhnd(enc, &mdk, dk, bh, n, D) ||
+        !encode_bhnd(enc, &mdv, dv, bh, n, D))
+        return ATTN_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0];
+        if (!set) {
+            int rc = prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
+            if (rc == ATTN_OK)
+                rc = prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+            if (rc != ATTN_OK) return rc;
+            set = true;
+        }
+    }
+    const BwdWorkspace w = workspace_layout(bh, n, D);
+    float *lse2 = reinterpret_cast<float *>(ws + w.acc_bytes);
+    float *delta = reinterpret_cast<float *>(ws + w.acc_bytes + w.stat_bytes);
+    const int n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
+
+    // 1. delta and lse2
+    const int64_t prep_threads = bh * n_pad * (D / 8);
+    const int64_t prep_blocks = (prep_threads + 255) / 256;
+    if (prep_blocks > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+    attn_sm100::attn_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, lse2, delta,
+        bh, n, n_pad);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    attn_sm100::BwdParams p;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.status = status;
+    p.n = n;
+    p.n_pad = n_pad;
+    p.num_k_tiles = (n + attn_sm100::BN - 1) / attn_sm100::BN;
+    p.num_q_tiles = (n + attn_sm100::BM - 1) / attn_sm100::BM;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal;
+    p.window = effective_window(n, window);
+
+    // 2. dK, dV: one CTA per key tile
+    attn_sm100::attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bh * p.num_k_tiles), KV::THREADS,
+                                          KV::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    // 3. dQ: one CTA per query tile
+    attn_sm100::attn_bwd_dq_kernel<D><<<static_cast<unsigned>(bh * p.num_q_tiles), QC::THREADS,
+                                        QC::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// The fused design: prep (delta, lse2, zeroed accumulator), one key-tile
+// kernel, accumulator -> bf16 dQ.
+template <int D>
+int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                     const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int n,
+                     float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+{
+    using Cfg = attn_sm100::FusedBwdCfg<D>;
     auto enc = encoder();
     if (!enc) return ATTN_ERR_CUDA;
     const int64_t bh = static_cast<int64_t>(B) * H;
@@ -85,16 +174,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         std::lock_guard<std::mutex> lk(g_mu);
         bool &set = g_bwd_set[dev][D == 128 ? 1 : 0];
         if (!set) {
-            // Same rule as the forward kernel: the register split between
-            // warpgroups needs exactly the per-thread count it was computed for.
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, attn_sm100::attn_bwd_kernel<D>) != cudaSuccess)
-                return ATTN_ERR_CUDA;
-            if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
-            if (cudaFuncSetAttribute(attn_sm100::attn_bwd_kernel<D>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Cfg::SMEM_BYTES) != cudaSuccess)
-                return ATTN_ERR_CUDA;
+            const int rc = prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH);
+            if (rc != ATTN_OK) return rc;
             set = true;
         }
     }
@@ -105,17 +186,15 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     float *delta = reinterpret_cast<float *>(ws + w.acc_bytes + w.stat_bytes);
     const int n_pad = (n + attn_sm100::BM - 1) / attn_sm100::BM * attn_sm100::BM;
 
-    // 1. delta, lse2, zeroed accumulator
     const int64_t prep_threads = bh * n_pad * (D / 8);
     const int64_t prep_blocks = (prep_threads + 255) / 256;
     if (prep_blocks > INT_MAX) return ATTN_ERR_UNSUPPORTED;
-    attn_sm100::attn_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
+    attn_sm100::attn_bwd_fused_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, lse2, delta,
         acc, bh, n, n_pad);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
-    // 2. main kernel
-    attn_sm100::BwdParams p;
+    attn_sm100::FusedBwdParams p;
     p.dq_acc = acc;
     p.lse2 = lse2;
     p.delta = delta;
@@ -128,11 +207,10 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.causal = causal;
     p.window = effective_window(n, window);
     const unsigned grid = static_cast<unsigned>(bh * p.num_k_tiles);
-    attn_sm100::attn_bwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
-                                                                                    mdv, macc, p);
+    attn_sm100::attn_bwd_fused_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
+                                                                                          mdv, macc, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
-    // 3. dQ accumulator -> bf16
     const int64_t count8 = bh * n * D / 8;
     const int64_t conv_blocks = (count8 + 255) / 256;
     if (conv_blocks > INT_MAX) return ATTN_ERR_UNSUPPORTED;
@@ -145,7 +223,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 
 extern "C" int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d)
 {
-    if (check_bwd_args(B, H, n, d, 1.f, 0, -1) != ATTN_OK) return -1;
+    if (check_bwd_args(B, H, n, d, 1.f, 0) != ATTN_OK) return -1;
     return static_cast<int64_t>(workspace_layout(static_cast<int64_t>(B) * H, n, d).total);
 }
 
@@ -155,7 +233,7 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
                         int window, void *stream)
 {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
-    const int rc = check_bwd_args(B, H, n, d, scale, causal, window);
+    const int rc = check_bwd_args(B, H, n, d, scale, causal);
     if (rc != ATTN_OK) return rc;
     for (const void *ptr : {q, k, v, o, dout, static_cast<const void *>(dq), static_cast<const void *>(dk),
                             static_cast<const void *>(dv), static_cast<const void *>(workspace)})
@@ -168,9 +246,9 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
     if (!status) return ATTN_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
-    if (d == 64)
-        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window, st,
-                              dev, status);
+    if (fused_for(d))
+        return launch_bwd_fused<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window,
+                                    st, dev, status);
     return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window, st, dev,
                            status);
 }

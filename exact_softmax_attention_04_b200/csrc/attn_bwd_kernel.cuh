@@ -12,39 +12,36 @@
 // delta_i equals sum_j P_ij dP_ij because O_i = sum_j P_ij v_j.
 //
 // Three launches on one stream:
-//   1. attn_bwd_prep_kernel: delta_i and LSE_i * log2(e) per row (padded to a
-//      whole number of 128-row tiles per head), and zeroes the fp32 dQ
-//      accumulator.
-//   2. attn_bwd_kernel: one CTA per (batch*head, 128-key tile). K_j and V_j
-//      stay in shared memory; the CTA walks the query tiles i that can attend
-//      to key tile j and, per tile, runs five tcgen05 MMAs:
-//        S^T  = K_j Q_i^T        (smem x smem -> TMEM, 128 keys x 128 queries)
-//        dP^T = V_j dO_i^T       (smem x smem -> TMEM)
-//        dV  += P^T dO_i         (P^T from TMEM, written there by the softmax warps)
-//        dK  += dS^T Q_i         (dS^T from shared memory, K-major)
-//        dQ_i = dS K_j           (the same dS buffer read MN-major)
-//      dK, dV accumulate in TMEM over the whole walk and are stored once;
-//      each dQ_i tile is added into the fp32 accumulator by TMA bulk
-//      reduce-adds from shared memory (several key tiles contribute to every
-//      query row).
-//   3. attn_bwd_dq_convert_kernel: fp32 dQ accumulator -> bf16 dQ.
+//   1. attn_bwd_prep_kernel: delta_i and LSE_i * log2(e) per row, padded to a
+//      whole number of 128-row tiles per head.
+//   2. attn_bwd_dkdv_kernel: one CTA per (batch*head, 128-key tile j). K_j,
+//      V_j stay in shared memory; the CTA walks the query tiles i that attend
+//      to tile j and runs, per query tile, four tcgen05 MMAs:
+//        S^T  = K_j Q_i^T   (smem x smem -> TMEM, 128 keys x 128 queries)
+//        dP^T = V_j dO_i^T  (smem x smem -> TMEM)
+//        dV  += P^T dO_i    (P^T in TMEM, over S^T's columns)
+//        dK  += dS^T Q_i    (dS^T in TMEM, over dP^T's columns)
+//      dV and dK accumulate in TMEM over the walk and are stored once.
+//   3. attn_bwd_dq_kernel: one CTA per (batch*head, 128-query tile i), Q_i
+//      and dO_i held in TMEM as MMA operands; it walks the key tiles j that
+//      tile i attends to and runs three MMAs per key tile:
+//        S  = Q_i K_j^T, dP = dO_i V_j^T   (TMEM x smem -> TMEM)
+//        dQ += dS K_j                      (dS in TMEM, over dP's columns)
+//      dQ accumulates in TMEM and is stored once.
+// Computing dQ in a kernel of its own costs two more MMAs per tile pair (S
+// and dP are recomputed) but needs no cross-CTA accumulation: adding each
+// (key tile, query tile) contribution to a global fp32 dQ, by atomics or by
+// TMA reduce-adds, was bound by the L2's reduction throughput (about
+// 2.7 TB/s measured) at well under half the tensor-core rate.
 //
-// Roles of the main kernel (512 threads, 16 warps = 4 warpgroups):
-//   warps 0-3, 4-7  "softmax": thread r of warpgroup h owns key row r (TMEM
-//                   lane r) and query columns [64h, 64h+64) of the tile. It
-//                   turns S^T into P^T (written back into TMEM over its own S
-//                   columns) and dP^T into dS^T (bf16, into the swizzled dS
-//                   buffer); after the walk it stores dV (h = 0) or dK (h = 1).
+// Roles of both main kernels (384 threads, 12 warps = 3 warpgroups):
+//   warps 0-3, 4-7  "softmax": warpgroup h owns TMEM lanes 0-127 (thread r,
+//                   lane r) and columns [64h, 64h+64) of the 128 x 128 tile.
 //   warp 8          MMA issuer (one elected lane) and TMEM owner.
-//   warp 9          TMA producer: K_j, V_j once, then Q_i, dO_i and the rows'
-//                   LSE and delta into a two-stage ring.
+//   warp 9          TMA producer.
 //   warps 10-11     idle.
-//   warps 12-15     dQ drain: TMEM -> registers (times scale) -> swizzled fp32
-//                   staging in shared memory -> TMA reduce-add into the
-//                   accumulator, 64 columns (32 KB) at a time.
-// Registers: launched at 128 per thread; the softmax warpgroups raise to 184,
-// the dQ warpgroup drops to 88 and the MMA/TMA warpgroup to 56
-// (2*184 + 88 + 56 = 4*128).
+// Registers: launched at 168 per thread; the softmax warpgroups raise to 232
+// and the third drops to 40 (2*128*232 + 128*40 = 384*168).
 //
 // Every wait is bounded as in the forward kernel: on expiry the kernel sets
 // bit 1 of the device status word, the other roles stop, copies and MMAs in
@@ -54,8 +51,6 @@
 
 namespace attn_sm100 {
 
-constexpr int BWD_NSTAGE = 2;              // Q_i / dO_i ring stages
-
 // Of every 16 pairs of P entries a softmax thread computes, the first
 // ATTN_BWD_EX2_EMU use the FMA-pipe polynomial for 2^x instead of the MUFU
 // (masked entries are zeroed after the exponential, so the polynomial's
@@ -63,71 +58,82 @@ constexpr int BWD_NSTAGE = 2;              // Q_i / dO_i ring stages
 #ifndef ATTN_BWD_EX2_EMU
 #define ATTN_BWD_EX2_EMU 2
 #endif
-constexpr int STATUS_SMEM_ALIGN = 2;       // device status bit: shared memory base not alignable
+constexpr int STATUS_SMEM_ALIGN = 2;  // device status bit: shared memory base not alignable
 
 struct BwdParams {
-    float *dq_acc;       // [B*H, n, d] fp32, zeroed by the prep kernel
     const float *lse2;   // [B*H, n_pad] LSE * log2(e)
     const float *delta;  // [B*H, n_pad] dO . O
     int *status;
     int n;
     int n_pad;           // n rounded up to a multiple of 128
     int num_k_tiles;     // ceil(n / 128)
+    int num_q_tiles;     // ceil(n / 128)
     float scale;         // softmax scale (factor of dQ and dK)
     float scale_log2;    // scale * log2(e)
     int causal;
     int window;          // < 0: none
 };
 
+// Launch shape shared by both main kernels.
+struct BwdRoles {
+    static constexpr int THREADS = 384;
+    static constexpr uint32_t REGS_LAUNCH = 168;
+    static constexpr uint32_t REGS_SOFTMAX = 232;
+    static constexpr uint32_t REGS_CTRL = 40;
+    static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_CTRL == THREADS * REGS_LAUNCH,
+                  "register split must use exactly the launch allocation");
+};
+
+// dK / dV kernel: K_j, V_j, a ring of NST (Q_i, dO_i, lse2_i, delta_i) stages.
 template <int D>
-struct BwdCfg {
+struct BwdKVCfg : BwdRoles {
     static_assert(D == 64 || D == 128, "head size 64 or 128");
     static constexpr int TILE_BYTES = BM * D * 2;
     static constexpr int BOXES = D / BOX_COLS;
-    static constexpr int NST = BWD_NSTAGE;
-    static constexpr int DS_BYTES = BN * BM * 2;  // 128 keys x 128 queries bf16
+    static constexpr int NST = (D == 128) ? 2 : 4;
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = K_OFF + TILE_BYTES;
-    static constexpr int Q_OFF = V_OFF + TILE_BYTES;        // + s * TILE_BYTES
+    static constexpr int Q_OFF = V_OFF + TILE_BYTES;         // + s * TILE_BYTES
     static constexpr int DO_OFF = Q_OFF + NST * TILE_BYTES;  // + s * TILE_BYTES
-    static constexpr int DS_OFF = DO_OFF + NST * TILE_BYTES;
-    static constexpr int STAT_OFF = DS_OFF + DS_BYTES;       // + s * 1024: lse2[128], delta[128]
-    // dQ staging for the TMA reduce-add: 64 fp32 columns of the 128 query
-    // rows (32 KB, two 128-byte swizzled boxes of 32 columns). D = 64 has a
-    // buffer of its own; D = 128 has no room left and stages its two halves
-    // in the dS buffer, which is idle from the end of dQ_i's MMA until the
-    // softmax writes dS_{i+1}.
-    static constexpr bool DQ_IN_DS = (D == 128);
-    static constexpr int DQS_HALF_BYTES = BM * 64 * 4;
-    static constexpr int DQS_OWN_OFF = STAT_OFF + NST * 1024;
-    static constexpr int BAR_OFF = DQS_OWN_OFF + (DQ_IN_DS ? 0 : DQS_HALF_BYTES);
-    static constexpr int DQS_OFF = DQ_IN_DS ? DS_OFF : DQS_OWN_OFF;
-    // kv_full, q_full[NST], q_empty[NST], s_full, dp_full, p_ready, ds_ready,
-    // dq_full, dq_free, ds_free, kv_done, drain, dqs_free
-    static constexpr int NUM_BARS = 11 + 2 * NST;
+    static constexpr int STAT_OFF = DO_OFF + NST * TILE_BYTES;  // + s * 1024: lse2[128], delta[128]
+    static constexpr int BAR_OFF = STAT_OFF + NST * 1024;
+    // kv_full, q_full[NST], q_empty[NST], s_full, dp_full, p_ready, ds_ready, kv_done, drain
+    static constexpr int NUM_BARS = 7 + 2 * NST;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
-    static constexpr int SMEM_USED = MISC_OFF + 16;
-    // Slack for aligning the dynamic shared memory base to 1024 bytes (the
-    // 128-byte swizzle atoms need it); at D = 128 less than 1 KB is left.
-    static constexpr int SLACK = (232448 - SMEM_USED >= 1024) ? 1024 : ((232448 - SMEM_USED) & ~127);
-    static constexpr int SMEM_BYTES = SMEM_USED + SLACK;
-    static_assert(SLACK >= 128 && SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + 1 KB alignment slack
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t S_COL = 0;     // S^T, then P^T in [0,32) and [64,96)
-    static constexpr uint32_t DP_COL = 128;  // dP^T
+    static constexpr uint32_t S_COL = 0;     // S^T; P^T over [0,32) and [64,96)
+    static constexpr uint32_t DP_COL = 128;  // dP^T; dS^T over [128,160) and [192,224)
     static constexpr uint32_t DV_COL = 256;
     static constexpr uint32_t DK_COL = 256 + D;
-    // dQ_i: D = 64 has columns of its own; D = 128 reuses dP^T's once the
-    // softmax warps have read dP^T.
-    static constexpr uint32_t DQ_COL = (D == 128) ? DP_COL : 256 + 2 * D;
-    static_assert(DQ_COL + D <= TMEM_COLS && DK_COL + D <= TMEM_COLS, "TMEM budget");
-    static constexpr int THREADS = 512;
-    static constexpr uint32_t REGS_LAUNCH = 128;
-    static constexpr uint32_t REGS_SOFTMAX = 184;
-    static constexpr uint32_t REGS_DQ = 88;
-    static constexpr uint32_t REGS_CTRL = 56;
-    static_assert(2 * REGS_SOFTMAX + REGS_DQ + REGS_CTRL == 4 * REGS_LAUNCH,
-                  "register split must use exactly the launch allocation");
+    static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
+};
+
+// dQ kernel: Q_i and dO_i (copied into TMEM at the start), then K_j, V_j
+// alternately in a ring of NSLOT tiles.
+template <int D>
+struct BwdQCfg : BwdRoles {
+    static_assert(D == 64 || D == 128, "head size 64 or 128");
+    static constexpr int TILE_BYTES = BM * D * 2;
+    static constexpr int BOXES = D / BOX_COLS;
+    static constexpr int NSLOT = (D == 128) ? 4 : 8;
+    static constexpr int Q_OFF = 0;    // also the dQ staging buffer of the epilogue
+    static constexpr int DO_OFF = TILE_BYTES;
+    static constexpr int KV_OFF = 2 * TILE_BYTES;  // + slot * TILE_BYTES
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // qd_full, qd_tmem, kv_full[NSLOT], kv_empty[NSLOT], s_full, s_read, dp_full, ds_ready, dq_done, drain
+    static constexpr int NUM_BARS = 8 + 2 * NSLOT;
+    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t S_COL = 0;
+    static constexpr uint32_t DP_COL = 128;  // dP; dS over [128,160) and [192,224)
+    static constexpr uint32_t DQ_COL = 256;
+    static constexpr uint32_t QA_COL = 256 + D;           // Q_i as MMA operand: D/2 columns
+    static constexpr uint32_t DOA_COL = 256 + D + D / 2;  // dO_i likewise
+    static_assert(DOA_COL + D / 2 <= TMEM_COLS, "TMEM budget");
 };
 
 // 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
@@ -143,19 +149,6 @@ __device__ __forceinline__ void bulk_load_if(uint32_t leader, uint32_t dst, cons
         : "memory");
 }
 
-// 3-D tiled reduce-add shared -> global (fp32 add in L2; rows outside the
-// tensor are skipped), tracked by the issuing thread's bulk async-groups.
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap *map, uint32_t src, int x, int y, int z)
-{
-    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
-                 " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
-// Wait until every bulk async-group of this thread has completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr)
 {
     float4 v;
@@ -165,16 +158,36 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr)
     return v;
 }
 
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// 2^x for the pair of P entries with index `pair` among a thread's 32 pairs
+// (the polynomial for the first ATTN_BWD_EX2_EMU of every 16).
+__device__ __forceinline__ void ex2_pair(int pair, float x0, float x1, float &e0, float &e1)
+{
+    if ((pair % 16) < ATTN_BWD_EX2_EMU) {
+        ex2_poly_x2(x0, x1, e0, e1);
+    } else {
+        e0 = ex2_approx(x0);
+        e1 = ex2_approx(x1);
+    }
+}
+
 // ---------------------------------------------------------------------------
-// 1. delta_i = dO_i . O_i (fp32 over the bf16 values), lse2_i = LSE_i log2(e)
-// for rows i < n of every head (0 in the padding rows up to n_pad), and a
-// zeroed dQ accumulator. D/8 lanes per row, 8 elements (16 bytes) per lane.
+// 1. delta_i = dO_i . O_i (fp32 over the bf16 values) and lse2_i = LSE_i log2(e)
+// for rows i < n of every head, 0 in the padding rows up to n_pad. D/8 lanes
+// per row, 8 elements (16 bytes) per lane.
 template <int D>
 __global__ void __launch_bounds__(256)
     attn_bwd_prep_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
                          const float *__restrict__ lse, float *__restrict__ lse2,
-                         float *__restrict__ delta, float *__restrict__ dq_acc, int64_t bh_count, int n,
-                         int n_pad)
+                         float *__restrict__ delta, int64_t bh_count, int n, int n_pad)
 {
     constexpr int L = D / 8;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -198,9 +211,6 @@ __global__ void __launch_bounds__(256)
             acc = fmaf(a.x, b.x, acc);
             acc = fmaf(a.y, b.y, acc);
         }
-        float4 *z = reinterpret_cast<float4 *>(dq_acc + off);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int w = L / 2; w >= 1; w /= 2) acc += __shfl_xor_sync(0xffffffffu, acc, w);
@@ -208,24 +218,6 @@ __global__ void __launch_bounds__(256)
         delta[row] = real ? acc : 0.f;
         lse2[row] = real ? lse[bh * n + i] * 1.4426950408889634f : 0.f;
     }
-}
-
-// ---------------------------------------------------------------------------
-// 3. dQ (bf16) = dQ accumulator (fp32, already scaled); 8 elements per thread.
-__global__ void __launch_bounds__(256)
-    attn_bwd_dq_convert_kernel(const float *__restrict__ dq_acc, __nv_bfloat16 *__restrict__ dq,
-                               int64_t count8)
-{
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (t >= count8) return;
-    const float4 a = reinterpret_cast<const float4 *>(dq_acc)[2 * t];
-    const float4 b = reinterpret_cast<const float4 *>(dq_acc)[2 * t + 1];
-    uint4 r;
-    r.x = pack_bf16x2(a.x, a.y);
-    r.y = pack_bf16x2(a.z, a.w);
-    r.z = pack_bf16x2(b.x, b.y);
-    r.w = pack_bf16x2(b.z, b.w);
-    reinterpret_cast<uint4 *>(dq)[t] = r;
 }
 
 // Query tiles [qlo, qhi) holding a query that attends to some key of the key
@@ -244,29 +236,37 @@ __device__ __forceinline__ void query_tile_range(int k0, int n, int causal, int 
     }
 }
 
-// ---------------------------------------------------------------------------
-// 2. The main backward kernel.
-template <int D>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
-    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                    const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p)
+// Dynamic shared memory base rounded up to 1 KB (the 128-byte swizzle atoms
+// need it); false if the slack does not allow it (never with the 1 KB of
+// slack both kernels request; the caller then returns before touching any
+// barrier or TMEM).
+__device__ __forceinline__ bool smem_base_1k(uint8_t *raw_ptr, uint32_t &base, uint8_t *&base_ptr)
 {
-    using C = BwdCfg<D>;
+    const uint32_t raw = smem_addr(raw_ptr);
+    base = (raw + 1023u) & ~1023u;
+    base_ptr = raw_ptr + (base - raw);
+    return base - raw <= 1024u;
+}
+
+// ---------------------------------------------------------------------------
+// 2. dK and dV.
+template <int D>
+__global__ void __launch_bounds__(BwdRoles::THREADS, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                         const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                         const BwdParams p)
+{
+    using C = BwdKVCfg<D>;
     constexpr int NST = C::NST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t raw = smem_addr(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    if (base - raw > static_cast<uint32_t>(C::SLACK)) {
-        // Cannot happen with a 1 KB-aligned dynamic shared memory base; every
-        // thread takes this branch alike, before any barrier or TMEM use.
+    uint32_t base;
+    uint8_t *base_ptr;
+    if (!smem_base_1k(smem_raw, base, base_ptr)) {
         if (threadIdx.x == 0) atomicOr(p.status, STATUS_SMEM_ALIGN);
         return;
     }
-    uint8_t *const base_ptr = smem_raw + (base - raw);
-
-    const uint32_t sK = base + C::K_OFF, sV = base + C::V_OFF, sDS = base + C::DS_OFF;
+    const uint32_t sK = base + C::K_OFF, sV = base + C::V_OFF;
     auto sQ = [&](int s) { return base + C::Q_OFF + s * C::TILE_BYTES; };
     auto sdO = [&](int s) { return base + C::DO_OFF + s * C::TILE_BYTES; };
     auto sStat = [&](int s) { return base + C::STAT_OFF + s * 1024; };
@@ -276,8 +276,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     auto q_empty = [&](int s) { return bars + 8u * (1 + NST + s); };
     const uint32_t s_full = bars + 8u * (1 + 2 * NST);
     const uint32_t dp_full = s_full + 8, p_ready = s_full + 16, ds_ready = s_full + 24;
-    const uint32_t dq_full = s_full + 32, dq_free = s_full + 40, ds_free = s_full + 48;
-    const uint32_t kv_done = s_full + 56, drain_bar = s_full + 64, dqs_free = s_full + 72;
+    const uint32_t kv_done = s_full + 32, drain_bar = s_full + 40;
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
@@ -303,12 +302,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         mbar_init(dp_full, 1);
         mbar_init(p_ready, 2 * BN);
         mbar_init(ds_ready, 2 * BN);
-        mbar_init(dq_full, 1);
-        mbar_init(dq_free, BM);
-        mbar_init(ds_free, 1);
         mbar_init(kv_done, 1);
         mbar_init(drain_bar, 1);
-        mbar_init(dqs_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -328,7 +323,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const Waiter wt{abort_flag, p.status};
 
-    if (warp >= 8 && warp < 12) {
+    if (warp >= 8) {
       regs_decrease<C::REGS_CTRL>();
       const uint32_t leader = elect_one();
       if (warp == 9) {
@@ -373,15 +368,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_t = idesc_bf16_f32(BN, BM, 0, 0);  // S^T, dP^T: both K-major
-        constexpr uint32_t idesc_acc = idesc_bf16_f32(BN, D, 0, 1); // dV, dK: A K-major, B MN-major
-        constexpr uint32_t idesc_dq = idesc_bf16_f32(BM, D, 1, 1);  // dQ: A and B MN-major
+        constexpr uint32_t idesc_acc = idesc_bf16_f32(BN, D, 0, 1); // dV, dK: A in TMEM, B MN-major
         bool ok = __all_sync(0xffffffffu, wt.wait(kv_full, 0));
         tc_fence_after();
         const uint64_t k_kmaj = smem_desc_sw128(sK, 16, 1024);
         const uint64_t v_kmaj = smem_desc_sw128(sV, 16, 1024);
-        const uint64_t k_mn = smem_desc_sw128(sK, BOX_BYTES, 1024);
-        const uint64_t ds_kmaj = smem_desc_sw128(sDS, 16, 1024);
-        const uint64_t ds_mn = smem_desc_sw128(sDS, BOX_BYTES, 1024);
         auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
             if (!__all_sync(0xffffffffu, wt.wait(bar, parity))) return false;
             tc_fence_after();
@@ -408,11 +399,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             mma_commit_if(leader, dp_full);
         };
         // Issue order: S(0), dP(0), then per query tile it
-        //   dV(it), S(it+1), dK(it), dQ(it), dP(it+1).
-        // S(it+1) overwrites P(it) in TMEM right behind dV(it), its reader
-        // (MMAs complete in issue order), so the softmax warps can start on
-        // tile it+1 as soon as they have produced dS(it), while the tensor
-        // core runs dK(it) and dQ(it).
+        //   dV(it), S(it+1), dK(it), dP(it+1).
+        // S(it+1) overwrites P^T(it) right behind dV(it), its reader, and
+        // dP(it+1) overwrites dS^T(it) right behind dK(it) (MMAs complete in
+        // issue order), so the softmax warps can start on tile it+1 as soon
+        // as they have produced dS^T(it).
         if (ok) ok = wait(q_full(0), 0);
         if (ok) {
             issue_s(0);
@@ -436,91 +427,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 if (!(ok = wait(q_full((it + 1) % NST), ((it + 1) / NST) & 1u))) break;
                 issue_s(it + 1);
             }
+            // dK += dS^T Q: dS^T in TMEM like P^T, in dP^T's columns
             if (!(ok = wait(ds_ready, it & 1u))) break;
-            if (D == 64 && it > 0 && !(ok = wait(dq_free, (it - 1) & 1u))) break;
-            // dK += dS^T Q: dS^T K-major (keys are rows), Q MN-major
 #pragma unroll
             for (int kk = 0; kk < BM / 16; ++kk) {
-                const uint64_t off = static_cast<uint64_t>(((kk / 4) * BOX_BYTES + (kk % 4) * 32) >> 4);
-                mma_bf16_ss_if(leader, tmem + C::DK_COL, ds_kmaj + off, q_mn + static_cast<uint64_t>(kk * 128),
-                               idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t dcol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+                mma_bf16_ts_if(leader, tmem + C::DK_COL, tmem + C::DP_COL + dcol,
+                               q_mn + static_cast<uint64_t>(kk * 128), idesc_acc,
+                               (it > 0 || kk > 0) ? 1u : 0u);
             }
-            // dQ_it = dS K: the same buffer read with queries as rows (MN-major)
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-                mma_bf16_ss_if(leader, tmem + C::DQ_COL, ds_mn + static_cast<uint64_t>(kk * 128),
-                               k_mn + static_cast<uint64_t>(kk * 128), idesc_dq, kk > 0 ? 1u : 0u);
-            mma_commit_if(leader, dq_full);
-            mma_commit_if(leader, ds_free);
             mma_commit_if(leader, q_empty(s));
-            if (it + 1 < nq) {
-                // with D = 128, dQ_it sits in dP's columns: the drain must have read it
-                if (D == 128 && !(ok = wait(dq_free, it & 1u))) break;
-                issue_dp(it + 1);
-            }
+            if (it + 1 < nq) issue_dp(it + 1);
         }
         if (ok) mma_commit_if(leader, kv_done);
         // Every MMA this warp issued must finish before TMEM is freed.
         mma_commit_if(leader, drain_bar);
         wt.drain(drain_bar, 0);
       }
-    } else if (warp >= 12) {
-        // ------------------------------------------------------------ dQ drain
-        regs_decrease<C::REGS_DQ>();
-        const int r = threadIdx.x % BM;  // query row in the tile == TMEM lane
-        const bool issuer = (r == 0);
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-        const float sc = p.scale;
-        const uint32_t stage = base + C::DQS_OFF;
-        // 32 columns of row r (times scale) into staging box b: 16-byte chunk
-        // j of the 128-byte row lands at chunk j ^ (r % 8), the 128-byte
-        // swizzle the tensor map uses.
-        auto stage32 = [&](const uint32_t (&v)[32], int b) {
-            const uint32_t rowp = stage + b * (BM * 128) + r * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t chunk = static_cast<uint32_t>(j) ^ static_cast<uint32_t>(r & 7);
-                st_shared_v4(rowp + chunk * 16, f2u(u2f(v[4 * j]) * sc), f2u(u2f(v[4 * j + 1]) * sc),
-                             f2u(u2f(v[4 * j + 2]) * sc), f2u(u2f(v[4 * j + 3]) * sc));
-            }
-        };
-        for (int it = 0; it < nq; ++it) {
-            // all four warps take the same decision (they meet at named
-            // barriers below)
-            if (!named_bar_and(3, BM, wt.wait(dq_full, it & 1u))) break;
-            tc_fence_after();
-            const int q0 = (qlo + it) * BM;
-#pragma unroll 1
-            for (int hf = 0; hf < D / 64; ++hf) {
-                uint32_t va[32], vb[32];
-                tmem_ld32(lane_base + C::DQ_COL + 64 * hf, va);
-                tmem_ld32(lane_base + C::DQ_COL + 64 * hf + 32, vb);
-                if (hf == D / 64 - 1) {
-                    // dQ_i is in registers: its TMEM columns may be reused
-                    tc_fence_before();
-                    mbar_arrive(dq_free);
-                }
-                // the previous reduce-add must have read the staging buffer
-                if (issuer) tma_store_wait_read0();
-                named_bar_sync(3, BM);
-                stage32(va, 0);
-                stage32(vb, 1);
-                fence_proxy_async_smem();
-                named_bar_sync(3, BM);
-                if (issuer) {
-                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, bh);
-                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, bh);
-                    tma_store_commit();
-                }
-            }
-            if (C::DQ_IN_DS && issuer) {
-                // the staging used the dS buffer: hand it back to the softmax
-                tma_store_wait_read0();
-                mbar_arrive(dqs_free);
-            }
-        }
-        // every reduce-add must be complete before the kernel ends
-        if (issuer) bulk_wait_all();
     } else {
         // ------------------------------------------------------------ softmax / dS
         regs_increase<C::REGS_SOFTMAX>();
@@ -541,7 +464,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             const bool need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
                                    (window >= 0 && q0 + BM - 1 > k0 + window) ||
                                    (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
-            int lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
+            const int lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
             int hi = min(BM - 1, n - 1 - q0);
             if (window >= 0) hi = min(hi, key + window - q0);
             if (key >= n) hi = -1;
@@ -560,20 +483,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                                              make_float2(sc, sc), make_float2(-l4.x, -l4.y));
                     const float2 x23 = ffma2(make_float2(u2f(sv[4 * g + 2]), u2f(sv[4 * g + 3])),
                                              make_float2(sc, sc), make_float2(-l4.z, -l4.w));
-                    // pairs 16*c2 + 2g and 16*c2 + 2g + 1 of the thread's 32
                     float e[4];
-                    if ((2 * g) % 16 < ATTN_BWD_EX2_EMU) {
-                        ex2_poly_x2(x01.x, x01.y, e[0], e[1]);
-                    } else {
-                        e[0] = ex2_approx(x01.x);
-                        e[1] = ex2_approx(x01.y);
-                    }
-                    if ((2 * g + 1) % 16 < ATTN_BWD_EX2_EMU) {
-                        ex2_poly_x2(x23.x, x23.y, e[2], e[3]);
-                    } else {
-                        e[2] = ex2_approx(x23.x);
-                        e[3] = ex2_approx(x23.y);
-                    }
+                    ex2_pair(16 * c2 + 2 * g, x01.x, x01.y, e[0], e[1]);
+                    ex2_pair(16 * c2 + 2 * g + 1, x23.x, x23.y, e[2], e[3]);
                     if (need_mask) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
@@ -586,7 +498,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                     pk[2 * g] = pack_bf16x2(e[0], e[1]);
                     pk[2 * g + 1] = pack_bf16x2(e[2], e[3]);
                 }
-                // P^T over this thread's own, already read, S columns
+                // P^T over this thread's own, already read, S^T columns
                 tmem_st16(lane_base + C::S_COL + 64 * h + 16 * c2, pk);
             }
             tmem_wait_st();
@@ -595,14 +507,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
             ok = __all_sync(0xffffffffu, wt.wait(dp_full, it & 1u));
             if (!ok) break;
-            if (it > 0) {
-                // dK_{i-1} and dQ_{i-1} must have read the dS buffer (and, at
-                // D = 128, the dQ drain must have finished staging in it)
-                ok = __all_sync(0xffffffffu, wt.wait(C::DQ_IN_DS ? dqs_free : ds_free, (it - 1) & 1u));
-                if (!ok) break;
-            }
             tc_fence_after();
-            const uint32_t row_addr = sDS + h * BOX_BYTES + r * 128;
 #pragma unroll
             for (int c2 = 0; c2 < 2; ++c2) {
                 const int cb = 64 * h + 32 * c2;
@@ -619,15 +524,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                     pk[2 * g] = pack_bf16x2(s01.x, s01.y);
                     pk[2 * g + 1] = pack_bf16x2(s23.x, s23.y);
                 }
-                // dS^T row r, query columns cb .. cb+31 of box h: 16-byte chunks
-                // 4*c2 .. 4*c2+3 of the row, 128-byte swizzled
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint32_t chunk = static_cast<uint32_t>(4 * c2 + q4) ^ static_cast<uint32_t>(r & 7);
-                    st_shared_v4(row_addr + chunk * 16, pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-                }
+                // dS^T over this thread's own, already read, dP^T columns
+                tmem_st16(lane_base + C::DP_COL + 64 * h + 16 * c2, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
@@ -660,6 +560,312 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             if (r == 0) {
                 const CUtensorMap *map = h ? &tmdK : &tmdV;
                 for (int b = 0; b < C::BOXES; ++b) tma_store_3d(map, stage + b * BOX_BYTES, b * BOX_COLS, k0, bh);
+                tma_store_commit();
+                tma_store_wait_read0();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ.
+template <int D>
+__global__ void __launch_bounds__(BwdRoles::THREADS, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p)
+{
+    using C = BwdQCfg<D>;
+    constexpr int NSLOT = C::NSLOT;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint32_t base;
+    uint8_t *base_ptr;
+    if (!smem_base_1k(smem_raw, base, base_ptr)) {
+        if (threadIdx.x == 0) atomicOr(p.status, STATUS_SMEM_ALIGN);
+        return;
+    }
+    const uint32_t sQ = base + C::Q_OFF, sdO = base + C::DO_OFF;
+    auto sKV = [&](int slot) { return base + C::KV_OFF + slot * C::TILE_BYTES; };
+    const uint32_t bars = base + C::BAR_OFF;
+    const uint32_t qd_full = bars, qd_tmem = bars + 8;
+    auto kv_full = [&](int slot) { return bars + 8u * (2 + slot); };
+    auto kv_empty = [&](int slot) { return bars + 8u * (2 + NSLOT + slot); };
+    const uint32_t s_full = bars + 8u * (2 + 2 * NSLOT);
+    const uint32_t s_read = s_full + 8, dp_full = s_full + 16, ds_ready = s_full + 24;
+    const uint32_t dq_done = s_full + 32, drain_bar = s_full + 40;
+    uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
+    volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
+
+    const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0);
+
+    // Work: query tiles of one head adjacent in blockIdx (K / V reuse in L2);
+    // within a head the late tiles (the most key tiles under a causal mask)
+    // first.
+    const int bh = blockIdx.x / p.num_q_tiles;
+    const int qt = p.num_q_tiles - 1 - static_cast<int>(blockIdx.x % p.num_q_tiles);
+    const int q0 = qt * BM;
+    const int n = p.n;
+    int jlo, jhi;
+    key_tile_range(q0, n, p.causal, p.window, jlo, jhi);
+    const int nkv = jhi - jlo;  // >= 1: key q0 is allowed for query q0
+
+    if (threadIdx.x == 0) {
+        mbar_init(qd_full, 1);
+        mbar_init(qd_tmem, 2 * BM);
+        for (int i = 0; i < NSLOT; ++i) {
+            mbar_init(kv_full(i), 1);
+            mbar_init(kv_empty(i), 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_read, 2 * BM);
+        mbar_init(dp_full, 1);
+        mbar_init(ds_ready, 2 * BM);
+        mbar_init(dq_done, 1);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9 && (threadIdx.x % 32) == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+        tma_prefetch_desc(&tmdQ);
+    }
+    if (warp == 8) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Waiter wt{abort_flag, p.status};
+
+    if (warp >= 8) {
+      regs_decrease<C::REGS_CTRL>();
+      const uint32_t leader = elect_one();
+      if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        mbar_arrive_expect_tx_if(leader, qd_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int b = 0; b < C::BOXES; ++b) {
+            tma_load_3d_if(leader, sQ + b * BOX_BYTES, &tmQ, qd_full, b * BOX_COLS, q0, bh);
+            tma_load_3d_if(leader, sdO + b * BOX_BYTES, &tmdO, qd_full, b * BOX_COLS, q0, bh);
+        }
+        // item i: K of key tile jlo + i/2 (i even) or V of it (i odd)
+        int issued = 0;
+        for (int i = 0; i < 2 * nkv; ++i) {
+            const int slot = i % NSLOT;
+            if (i >= NSLOT &&
+                !__all_sync(0xffffffffu, wt.wait(kv_empty(slot), ((i / NSLOT) & 1u) ^ 1u)))
+                break;
+            mbar_arrive_expect_tx_if(leader, kv_full(slot), C::TILE_BYTES);
+            const CUtensorMap *map = (i & 1) ? &tmV : &tmK;
+            const int k0 = (jlo + i / 2) * BN;
+#pragma unroll
+            for (int b = 0; b < C::BOXES; ++b)
+                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
+            ++issued;
+        }
+        wt.drain(qd_full, 0);
+        for (int slot = 0; slot < NSLOT; ++slot)
+            if (issued > slot) wt.drain(kv_full(slot), ((issued - 1 - slot) / NSLOT) & 1u);
+      } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);  // S, dP: A in TMEM, B K-major
+        constexpr uint32_t idesc_dq = idesc_bf16_f32(BM, D, 0, 1);  // dQ: A in TMEM, B MN-major
+        auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+            if (!__all_sync(0xffffffffu, wt.wait(bar, parity))) return false;
+            tc_fence_after();
+            return true;
+        };
+        // ring item of K_t (2t) or V_t (2t + 1): its slot and the parity of its load
+        auto slot_of = [&](int item) { return item % NSLOT; };
+        auto par_of = [&](int item) { return static_cast<uint32_t>((item / NSLOT) & 1); };
+        // S(t) = Q K_t^T: A = Q from TMEM (D/2 columns, 8 per 16-wide K step)
+        auto issue_s = [&](int t) -> bool {
+            const int ik = 2 * t;
+            if (!wait(kv_full(slot_of(ik)), par_of(ik))) return false;
+            const uint64_t kdesc = smem_desc_sw128(sKV(slot_of(ik)), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                mma_bf16_ts_if(leader, tmem + C::S_COL, tmem + C::QA_COL + k * 8, kdesc + off, idesc_s,
+                               k > 0 ? 1u : 0u);
+            }
+            mma_commit_if(leader, s_full);
+            return true;
+        };
+        // dP(t) = dO V_t^T
+        auto issue_dp = [&](int t) -> bool {
+            const int iv = 2 * t + 1;
+            if (!wait(kv_full(slot_of(iv)), par_of(iv))) return false;
+            const uint64_t vdesc = smem_desc_sw128(sKV(slot_of(iv)), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                mma_bf16_ts_if(leader, tmem + C::DP_COL, tmem + C::DOA_COL + k * 8, vdesc + off, idesc_s,
+                               k > 0 ? 1u : 0u);
+            }
+            mma_commit_if(leader, dp_full);
+            return true;
+        };
+        // Issue order: S(0), dP(0), then per key tile t
+        //   S(t+1) once the softmax has read S(t); dQ(t), dP(t+1) once dS(t) is in TMEM.
+        // dS(t) sits in dP's columns; dP(t+1) overwrites it right behind
+        // dQ(t), its reader (MMAs complete in issue order).
+        bool ok = wait(qd_tmem, 0);
+        if (ok) ok = issue_s(0);
+        if (ok) ok = issue_dp(0);
+        for (int t = 0; ok && t < nkv; ++t) {
+            if (t + 1 < nkv) {
+                if (!(ok = wait(s_read, t & 1u))) break;
+                if (!(ok = issue_s(t + 1))) break;
+            }
+            if (!(ok = wait(ds_ready, t & 1u))) break;
+            // dQ += dS K_t: dS of keys [0,64) in TMEM columns [128,160), of
+            // keys [64,128) in [192,224); K_t read MN-major (keys along K)
+            const int ik = 2 * t;
+            const uint64_t kmn = smem_desc_sw128(sKV(slot_of(ik)), BOX_BYTES, 1024);
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+                const uint32_t dcol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+                mma_bf16_ts_if(leader, tmem + C::DQ_COL, tmem + C::DP_COL + dcol,
+                               kmn + static_cast<uint64_t>(kk * 128), idesc_dq, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_if(leader, kv_empty(slot_of(ik)));
+            mma_commit_if(leader, kv_empty(slot_of(ik + 1)));
+            if (t + 1 < nkv && !(ok = issue_dp(t + 1))) break;
+        }
+        if (ok) mma_commit_if(leader, dq_done);
+        mma_commit_if(leader, drain_bar);
+        wt.drain(drain_bar, 0);
+      }
+    } else {
+        // ------------------------------------------------------------ softmax / dS
+        regs_increase<C::REGS_SOFTMAX>();
+        const int h = warp / 4;                 // key columns [64h, 64h + 64)
+        const int r = threadIdx.x % BM;         // query row in the tile == TMEM lane
+        const int row = q0 + r;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+        const float sc = p.scale_log2;
+        const int causal = p.causal, window = p.window;
+        // this row's log2-domain LSE and delta (0 in rows past n)
+        const size_t srow = static_cast<size_t>(bh) * p.n_pad + row;
+        const float nl2 = -p.lse2[srow];
+        const float dlt = p.delta[srow];
+        // Q (h = 0) or dO (h = 1) row r -> TMEM as the A operand of S or dP:
+        // lane r, two bf16 per column, read out of the 128-byte swizzled tile.
+        bool ok = __all_sync(0xffffffffu, wt.wait(qd_full, 0));
+        if (ok) {
+            const uint32_t src = h ? sdO : sQ;
+            const uint32_t dst = lane_base + (h ? C::DOA_COL : C::QA_COL);
+#pragma unroll
+            for (int b = 0; b < C::BOXES; ++b) {
+                uint32_t v[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t chunk = static_cast<uint32_t>(j) ^ static_cast<uint32_t>(r & 7);
+                    const uint4 u = ld_shared_u4(src + b * BOX_BYTES + r * 128 + chunk * 16);
+                    v[4 * j] = u.x;
+                    v[4 * j + 1] = u.y;
+                    v[4 * j + 2] = u.z;
+                    v[4 * j + 3] = u.w;
+                }
+                tmem_st32(dst + b * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(qd_tmem);
+        }
+        for (int t = 0; ok && t < nkv; ++t) {
+            const int k0 = (jlo + t) * BN;
+            ok = __all_sync(0xffffffffu, wt.wait(s_full, t & 1u));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sa[32], sb[32];
+            tmem_ld32(lane_base + C::S_COL + 64 * h, sa);
+            tmem_ld32(lane_base + C::S_COL + 64 * h + 32, sb);
+            // S(t) is in registers: the MMA warp may compute S(t+1)
+            tc_fence_before();
+            mbar_arrive(s_read);
+            const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
+                                   (window >= 0 && k0 < q0 + BM - 1 - window) ||
+                                   (!causal && window >= 0 && k0 + BN - 1 > q0 + window);
+            // allowed key columns of this row: [lo, hi], key = k0 + column
+            const int hi = min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1), n - 1 - k0);
+            const int lo = (window >= 0) ? row - window - k0 : 0;
+            float pf[64];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t s0 = (i < 16) ? sa[2 * i] : sb[2 * i - 32];
+                const uint32_t s1 = (i < 16) ? sa[2 * i + 1] : sb[2 * i - 31];
+                const float2 x = ffma2(make_float2(u2f(s0), u2f(s1)), make_float2(sc, sc), make_float2(nl2, nl2));
+                ex2_pair(i, x.x, x.y, pf[2 * i], pf[2 * i + 1]);
+            }
+            if (need_mask) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int c = 64 * h + i;
+                    if (c < lo || c > hi) pf[i] = 0.f;
+                }
+            }
+            ok = __all_sync(0xffffffffu, wt.wait(dp_full, t & 1u));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                uint32_t dv[32];
+                tmem_ld32(lane_base + C::DP_COL + 64 * h + 32 * c2, dv);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 tt = fsub2(make_float2(u2f(dv[2 * i]), u2f(dv[2 * i + 1])), make_float2(dlt, dlt));
+                    const float2 ds = fmul2(tt, make_float2(pf[32 * c2 + 2 * i], pf[32 * c2 + 2 * i + 1]));
+                    pk[i] = pack_bf16x2(ds.x, ds.y);
+                }
+                // dS over this thread's own, already read, dP columns
+                tmem_st16(lane_base + C::DP_COL + 64 * h + 16 * c2, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ds_ready);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, wt.wait(dq_done, 0));
+        const bool all_ok = named_bar_and(1, 2 * BM, ok);
+        if (all_ok) {
+            tc_fence_after();
+            // scale * dQ: warpgroup h stores columns [h*D/2, (h+1)*D/2) of row
+            // r -> bf16 -> swizzled smem (the Q tile, unused since it was
+            // copied into TMEM) -> TMA store; rows past n are clipped.
+            const float mul = p.scale;
+#pragma unroll 1
+            for (int c = h * (D / 2); c < (h + 1) * (D / 2); c += 32) {
+                uint32_t v[32];
+                tmem_ld32(lane_base + C::DQ_COL + c, v);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(u2f(v[2 * i]) * mul, u2f(v[2 * i + 1]) * mul);
+                const uint32_t rowp = sQ + (c / BOX_COLS) * BOX_BYTES + r * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t chunk = static_cast<uint32_t>((c % BOX_COLS) / 8 + q4) ^ static_cast<uint32_t>(r & 7);
+                    st_shared_v4(rowp + chunk * 16, pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 2 * BM);
+            if (threadIdx.x == 0) {
+                for (int b = 0; b < C::BOXES; ++b) tma_store_3d(&tmdQ, sQ + b * BOX_BYTES, b * BOX_COLS, q0, bh);
                 tma_store_commit();
                 tma_store_wait_read0();
             }

@@ -189,16 +189,21 @@ ATTN_API int attn_fwd_host_noalloc(const void *q, const void *k, const void *v, 
  *   dq, dk, dv       : device, bf16 [B, H, n, d], 16-byte aligned, written
  *   workspace        : device scratch owned by the caller, 16-byte aligned,
  *                      at least attn_bwd_workspace_bytes(B, H, n, d) bytes
- *                      (an fp32 dQ accumulator and two fp32 per-row arrays);
+ *                      (two fp32 per-row arrays and, for d = 64, an fp32 dQ
+ *                      accumulator of 4 * B*H*n*d bytes);
  *                      its contents on entry do not matter, and it must not
  *                      be used by other work until this call's work is done
  *   B, H, n, d, scale, causal, window, stream : as attn_fwd (K and V have H
  *                      heads: the grouped-query form has no backward here)
  *
  * Arithmetic: bf16 tensor-core products with fp32 accumulation; P and dS
- * are rounded to bf16 before their products; dQ is accumulated in fp32 over
- * key tiles (atomic adds, so its last bits may differ between runs); dQ, dK,
- * dV are rounded to bf16 once. Three kernels are enqueued on `stream`.
+ * are rounded to bf16 before their products; all sums are fp32 and each
+ * gradient is rounded to bf16 once. d = 128: three kernels (per-row terms;
+ * dK and dV, one CTA per key tile; dQ, one CTA per query tile), results
+ * identical from run to run. d = 64: three kernels (per-row terms and a
+ * zeroed accumulator; one CTA per key tile computing dK, dV and adding its
+ * dQ contributions into the fp32 accumulator by bulk reduce-adds, whose
+ * order varies, so dQ's last bits may differ between runs; dQ conversion).
  * Returns as attn_fwd; ATTN_ERR_INVALID also for a short or misaligned
  * workspace. Outputs must not overlap inputs or the workspace.
  */

@@ -151,12 +151,12 @@ def test_attn_bwd_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
 
 
 def test_bwd_workspace_size(attn):
-    # fp32 dQ accumulator + two fp32 per-row arrays padded to 128-row tiles,
-    # each part rounded up to 256 bytes
+    # two fp32 per-row arrays padded to 128-row tiles, plus at d = 64 an fp32
+    # dQ accumulator, each part rounded up to 256 bytes
     def expect(B, H, n, d):
         r = lambda x: (x + 255) // 256 * 256
         n_pad = (n + 127) // 128 * 128
-        return r(B * H * n * d * 4) + 2 * r(B * H * n_pad * 4)
+        return (r(B * H * n * d * 4) if d == 64 else 0) + 2 * r(B * H * n_pad * 4)
     for shape in [(1, 1, 1, 64), (1, 2, 300, 64), (2, 3, 129, 128), (8, 8, 8192, 64)]:
         assert attn.bwd_workspace_bytes(*shape) == expect(*shape)
     assert attn.lib().attn_bwd_workspace_bytes(1, 1, 128, 80) == -1
