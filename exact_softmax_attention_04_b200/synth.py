@@ -158,6 +158,71 @@ GQA_N8192 = Workload("B1-H64-Hkv8-n8192-d128-causal", 1, 64, 8192, 128, True, Hk
 SYM_N16384 = Workload("B2-H16-n16384-d64-symwindow256", 2, 16, 16384, 64, False, 256)
 
 
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """One decode step against rolling key/value caches of W slots: one query
+    token per sequence at position `pos` (every sequence at the same
+    position), grouped-query heads."""
+
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    W: int
+    d: int
+    pos: int
+    q_std: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def keys(self) -> int:
+        """Cached positions each query attends to."""
+        return min(self.pos + 1, self.W)
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "B": self.B, "H": self.H, "H_kv": self.Hkv, "cache_slots": self.W,
+                "d": self.d, "position": self.pos, "keys_per_query": self.keys,
+                "scale": f"1/sqrt({self.d})", "q_std": self.q_std, "seed": self.seed}
+
+
+def make_decode(B: int, H: int, Hkv: int, W: int, d: int, seed: int = 0, q_std: float = 1.0
+                ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """q [B, H, d] and rolling caches k, v [B, Hkv, W, d], bf16, drawn like
+    make_qkv (q, then k, then v from one generator seeded `seed`)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, d), generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q.mul_(q_std)
+    k = torch.randn((B, Hkv, W, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, W, d), generator=g, dtype=torch.float32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def ring_from_sequence(seq: torch.Tensor, W: int) -> torch.Tensor:
+    """The rolling cache after writing positions 0 .. T-1 of `seq` [B, Hkv,
+    T, d] in order, position p into slot p mod W (unwritten slots zero)."""
+    B, Hkv, T, d = seq.shape
+    ring = torch.zeros((B, Hkv, W, d), dtype=seq.dtype)
+    for p in range(T):
+        ring[:, :, p % W] = seq[:, :, p]
+    return ring
+
+
+# Decode against a 4096-slot rolling cache at position 32767 (n = 32,768, the
+# worked example's cache size), Mistral-7B-like heads (32 query heads sharing
+# 8 key/value heads, d = 128), 64 sequences per step.
+DECODE_W4096 = DecodeWorkload("decode-B64-H32-Hkv8-W4096-d128-pos32767", 64, 32, 8, 4096, 128, 32767)
+
+
+def decode_by_name(name: str) -> Optional[DecodeWorkload]:
+    return DECODE_W4096 if name == DECODE_W4096.name else None
+
+
 def sweep() -> List[Workload]:
     """n in {1024, 4096, 16384, 65536} x d in {64, 128} x five masks;
     B*H*n = 262144 tokens (B=1); Q ~ N(0, 4^2) for large logits."""

@@ -58,6 +58,8 @@ def _load():
         lib.oracle_attn_bwd_rows_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
                                                  i64, vp, i64, vp, i64, vp, vp, vp]
         lib.oracle_attn_bwd_rows_f64.restype = ip
+        lib.oracle_attn_decode_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp]
+        lib.oracle_attn_decode_f64.restype = ip
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ip
         _lib = lib
@@ -185,6 +187,30 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, window: int = -1
     rows = np.arange(B * H * n, dtype=np.int64)
     dq, dk, dv = attn_bwd_rows(q, k, v, dout, scale, causal, window, rows, rows)
     return dq.reshape(B, H, n, d), dk.reshape(B, H, n, d), dv.reshape(B, H, n, d)
+
+
+def attn_decode(q, k_cache, v_cache, pos, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode against rolling caches: q bf16 [B, H, d], k_cache / v_cache bf16
+    [B, Hkv, W, d] (position p at slot p mod W), pos [B] (>= 0). Returns O
+    [B, H, d] and LSE [B, H] in fp64."""
+    lib = _load()
+    if len(q.shape) != 3 or len(k_cache.shape) != 4 or k_cache.shape != v_cache.shape:
+        raise ValueError("q must be [B, H, d] and the caches [B, Hkv, W, d]")
+    B, H, d = q.shape
+    Bk, Hkv, W, dk = k_cache.shape
+    if Bk != B or dk != d:
+        raise ValueError("cache shape does not match q")
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    if p.size != B:
+        raise ValueError("pos must have B entries")
+    o = np.empty((B, H, d), dtype=np.float64)
+    lse = np.empty((B, H), dtype=np.float64)
+    rc = lib.oracle_attn_decode_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, p.ctypes.data,
+                                    B, H, Hkv, W, d, float(scale), o.ctypes.data, lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_decode_f64 rejected its arguments (rc={rc})")
+    return o, lse
 
 
 def matmul(a: np.ndarray, b: np.ndarray, ta: bool = False, tb: bool = False) -> np.ndarray:

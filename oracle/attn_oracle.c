@@ -477,3 +477,81 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
     free(rowterm);
     return bad ? 2 : 0;
 }
+
+/* ========================================================================
+ * Decode against a rolling key/value cache.
+ *
+ * One query token per sequence attends to the keys a sliding window keeps.
+ * The cache is the rolling buffer of "Sparse & sub-quadratic attention"
+ * (worked example of the maths panel: a 4,096-position cache serving
+ * n = 32,768, after Mistral): W slots per key/value head, position p stored
+ * at slot p mod W, so after writing position t the cache holds positions
+ * max(0, t - W + 1) .. t. For sequence b with query position t = pos[b] and
+ * query head h (key/value head h / (H / Hkv), as for grouped-query
+ * attention) the output is the plain definition over those positions:
+ *   s_p  = scale * q . k(slot p mod W),  M = max_p s_p,
+ *   O    = sum_p exp(s_p - M) v(slot p mod W) / sum_p exp(s_p - M),
+ *   LSE  = M + ln sum_p exp(s_p - M).
+ *   q      : bf16 [B, H, d];  k, v : bf16 [B, Hkv, W, d];  pos : int64 [B], >= 0
+ *   o      : fp64 [B, H, d];  lse : fp64 [B, H]
+ * ======================================================================== */
+int oracle_attn_decode_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int64_t *pos,
+                           int64_t B, int64_t H, int64_t Hkv, int64_t W, int64_t d, double scale,
+                           double *o, double *lse)
+{
+    if (!q || !k || !v || !pos || !o || !lse || B <= 0 || H <= 0 || Hkv <= 0 || W <= 0 || d <= 0)
+        return 1;
+    if (H % Hkv != 0)
+        return 1;
+    for (int64_t b = 0; b < B; ++b)
+        if (pos[b] < 0)
+            return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)W);
+        if (!s) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t bh = 0; bh < B * H; ++bh) {
+                const int64_t b = bh / H, h = bh % H;
+                const int64_t kvh = b * Hkv + h / (H / Hkv);
+                const int64_t t = pos[b];
+                const int64_t first = (t - W + 1 > 0) ? t - W + 1 : 0;
+                const int64_t count = t - first + 1;
+                const uint16_t *qh = q + bh * d;
+                /* pass 1: scores of the cached positions and their maximum */
+                double M = -INFINITY;
+                for (int64_t u = 0; u < count; ++u) {
+                    const int64_t slot = (first + u) % W;
+                    const uint16_t *kr = k + (kvh * W + slot) * d;
+                    double acc = 0.0;
+                    for (int64_t c = 0; c < d; ++c)
+                        acc += bf16_to_f64(qh[c]) * bf16_to_f64(kr[c]);
+                    s[u] = scale * acc;
+                    if (s[u] > M)
+                        M = s[u];
+                }
+                /* pass 2: normaliser and weighted sum of values */
+                double Z = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    o[bh * d + c] = 0.0;
+                for (int64_t u = 0; u < count; ++u) {
+                    const int64_t slot = (first + u) % W;
+                    const uint16_t *vr = v + (kvh * W + slot) * d;
+                    const double w = exp(s[u] - M);
+                    Z += w;
+                    for (int64_t c = 0; c < d; ++c)
+                        o[bh * d + c] += w * bf16_to_f64(vr[c]);
+                }
+                for (int64_t c = 0; c < d; ++c)
+                    o[bh * d + c] /= Z;
+                lse[bh] = M + log(Z);
+            }
+        }
+        free(s);
+    }
+    return bad ? 2 : 0;
+}
