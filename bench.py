@@ -515,6 +515,103 @@ def run_bwd(args, wl, world, rank, local):
     return 0
 
 
+DECODE_METRIC = "decode GB/s (cached K and V read once, plus q, O, LSE)"
+
+
+def run_decode(args, wl, world, rank, local):
+    """One decode step against rolling caches (attn_decode: split kernel and
+    merge) per step, timed like the forward; the roofline is HBM bandwidth on
+    the algorithmic bytes: the cached keys and values each query group
+    attends to, read once, plus q, O and LSE."""
+    import numpy as np
+    import exact_softmax_attention_04_b200 as attn
+    from exact_softmax_attention_04_b200 import synth
+
+    dev = torch.device("cuda", local)
+    q, kc, vc = synth.make_decode(wl.B, wl.H, wl.Hkv, wl.W, wl.d, seed=wl.seed, q_std=wl.q_std)
+    qd, kd, vd = q.to(dev), kc.to(dev), vc.to(dev)
+    pos = torch.full((wl.B,), wl.pos, dtype=torch.int32, device=dev)
+    o = torch.empty_like(qd)
+    lse = torch.empty((wl.B, wl.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(wl.B, wl.H, wl.Hkv, wl.W, wl.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = 2 * wl.B * wl.Hkv * wl.keys * wl.d * 2 + 2 * q.numel() * 2 + lse.numel() * 4
+    flops = 4 * wl.d * wl.keys * wl.B * wl.H
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        attn.attn_decode(qd, kd, vd, pos, wl.scale, out=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local if not args.profile else -1) as clocks:
+        if not args.profile:
+            time.sleep(0.5)
+        wall0 = time.time()
+        for i in range(args.steps):
+            flush.zero_()  # the caches (1.07 GB) exceed L2 anyway; flush so q/O do not linger
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        wall1 = time.time()
+    barrier(world)
+    st = attn.sync_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(attn.strerror(st))
+    times = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(statistics.mean(times), world)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": wl.name, "pass": "decode", "ms_per_step": ms, "gbs": gbs}),
+                  flush=True)
+        return 0
+    if rank != 0:
+        return 0
+    _, hbm_peak, peak_src = peaks()
+    line = {
+        "metric": DECODE_METRIC, "value": world * gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**wl.describe(), "pass": "decode",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed (256 MB write) before each timed step; the caches exceed L2"},
+        "tflops": flops / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": gbs / hbm_peak, "traffic": None, "peak_source": f"{peak_src} HBM copy",
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "note": "achieved over the attn_decode call (split kernel and merge kernel)"},
+        "e2e": {"value": None, "unit": "GB/s", "note": "decode has no host-buffer entry point"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(wall0, wall1),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        g = torch.Generator().manual_seed(2)
+        nseq = max(1, min(wl.B, 4))
+        t0 = time.perf_counter()
+        o_ref, lse_ref = oracle.attn_decode(q[:nseq], kc[:nseq], vc[:nseq], [wl.pos] * nseq, wl.scale)
+        dt = time.perf_counter() - t0
+        og = o[:nseq].float().cpu().numpy()
+        line["cpu_baseline"] = {
+            "value": nbytes * nseq / wl.B / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"the first {nseq} sequences of {wl.name}, fp64 oracle",
+            "parity_vs_gpu": {"o_max_abs": float(np.abs(og - o_ref).max()),
+                              "lse_max_abs": float(np.abs(lse[:nseq].cpu().numpy() - lse_ref).max())}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """Kernel time of every target workload (one line each): TFLOP/s on
     unmasked FLOPs, % of the measured peak and HBM GB/s on the minimum bytes
@@ -571,6 +668,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every target workload (kernel only, median of --steps, L2 flushed)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decode step against rolling caches (attn_decode); --workload "
+                         "defaults to decode-B64-H32-Hkv8-W4096-d128-pos32767")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (attn_bwd) of --workload instead of the forward")
     ap.add_argument("--profile", action="store_true",
@@ -582,6 +682,18 @@ def main():
     if args.sweep:
         return run_sweep(args)
     from exact_softmax_attention_04_b200 import synth
+    if args.decode:
+        name = args.workload if args.workload.startswith("decode-") else synth.DECODE_W4096.name
+        dwl = synth.decode_by_name(name)
+        if dwl is None:
+            raise SystemExit(f"unknown decode workload {name}")
+        world, rank, local = dist_setup(args.gpus)
+        try:
+            return run_decode(args, dwl, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
     wl = synth.by_name(args.workload)
     if wl is None:
         raise SystemExit(f"unknown workload {args.workload}")

@@ -1,6 +1,7 @@
 /*
  * attn.h - C ABI of the B200 (sm_100a) exact softmax attention library
- * (libattn_b200.so): forward pass, grouped-query forward, backward pass.
+ * (libattn_b200.so): forward pass, grouped-query forward, backward pass,
+ * decode against rolling key/value caches.
  *
  * The operation (all entry points that compute):
  *
@@ -215,6 +216,49 @@ ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o
 /* Device workspace bytes attn_bwd needs for this shape, or -1 if the shape
  * is invalid or unsupported. */
 ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
+
+/*
+ * attn_decode - one decode step against rolling key/value caches.
+ *
+ * Every sequence b has one new query token at position pos[b] (>= 0). Its
+ * keys and values live in a rolling cache of W slots per key/value head:
+ * position p is stored in slot p mod W, so after the current token's own
+ * key and value have been written the cache holds positions
+ * max(0, pos[b] - W + 1) .. pos[b] (the rolling buffer of the worked example
+ * on "Sparse & sub-quadratic attention": a 4,096-position cache serving
+ * n = 32,768). The query attends to exactly those positions:
+ *
+ *   O[b,h]   = softmax(scale * q[b,h] . k) v   over the cached positions,
+ *   LSE[b,h] = ln sum exp(scale * q[b,h] . k)  (natural-log units),
+ *
+ * with key/value head h / (H / Hkv) (grouped-query attention; Hkv = H for
+ * multi-head attention). This equals row pos[b] of attn_fwd with causal = 1
+ * and window = W - 1 over the sequence that filled the cache.
+ *
+ *   q                : device, bf16 [B, H, d], 16-byte aligned
+ *   k_cache, v_cache : device, bf16 [B, Hkv, W, d], 16-byte aligned, read only
+ *   pos              : device, int32 [B], read by the kernel (so a step can be
+ *                      enqueued without the host knowing the positions)
+ *   o, lse           : device, bf16 [B, H, d] and fp32 [B, H], written
+ *   workspace        : device scratch owned by the caller, 16-byte aligned,
+ *                      at least attn_decode_workspace_bytes(...) bytes
+ *                      (per-split partial results)
+ *   H / Hkv          : 1, 2, 4 or 8 (else ATTN_ERR_UNSUPPORTED); d: 64 or 128
+ *   B * Hkv          : at most 65535
+ *   scale, stream    : as attn_fwd
+ *
+ * A negative pos[b] is read as 0. Arithmetic: fp32 scores, softmax and
+ * accumulation on the CUDA cores over the bf16 inputs, O rounded to bf16.
+ * Two kernels are enqueued: per (split of the slots, sequence, kv head)
+ * partial results, then their log-sum-exp merge. Returns as attn_fwd.
+ */
+ATTN_API int attn_decode(const void *q, const void *k_cache, const void *v_cache, const int *pos,
+                         void *o, float *lse, void *workspace, size_t workspace_bytes, int B,
+                         int H, int Hkv, int W, int d, float scale, void *stream);
+
+/* Device workspace bytes attn_decode needs, or -1 if the shape is invalid
+ * or unsupported. */
+ATTN_API int64_t attn_decode_workspace_bytes(int B, int H, int Hkv, int W, int d);
 
 /*
  * attn_sync_status - synchronize `stream`, then read and clear this device's

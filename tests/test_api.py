@@ -169,3 +169,31 @@ def test_bwd_binding_checks_tensors_before_calling(attn):
     lse = torch.zeros(1, 1, 8)
     with pytest.raises(ValueError):
         attn.attn_bwd(q, q, q, q, lse, q)  # host tensors
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), 1), (dict(pos=0), 1), (dict(workspace=0), 1), (dict(B=0), 1), (dict(W=0), 1),
+    (dict(scale=0.0), 1), (dict(Hkv=3), 1), (dict(q=FAKE + 8), 1), (dict(pos=FAKE + 2), 1),
+    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(H=24, Hkv=2), 2), (dict(H=16, Hkv=1), 2),
+    (dict(B=70000, H=8, Hkv=1), 2),
+])
+def test_attn_decode_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, o=FAKE, lse=FAKE, workspace=FAKE, ws_bytes=1 << 40,
+             B=2, H=8, Hkv=2, W=4096, d=128, scale=0.125, stream=None)
+    a.update(kw)
+    rc = attn.lib().attn_decode(a["q"], a["k"], a["v"], a["pos"], a["o"], a["lse"], a["workspace"],
+                                a["ws_bytes"], a["B"], a["H"], a["Hkv"], a["W"], a["d"], a["scale"],
+                                a["stream"])
+    assert rc == code
+
+
+def test_decode_workspace_size(attn):
+    # per-split partials: nsplit * B * H * (d + 2) fp32, nsplit from the split rule
+    def expect(B, H, Hkv, W, d):
+        tiles = (W + 63) // 64
+        ns = max(1, min(tiles, (4 * 148 + B * Hkv - 1) // (B * Hkv)))
+        chunk = ((tiles + ns - 1) // ns) * 64
+        return ((W + chunk - 1) // chunk) * B * H * (d + 2) * 4
+    for shape in [(1, 1, 1, 1, 64), (2, 8, 2, 4096, 128), (64, 32, 8, 4096, 128), (3, 4, 4, 200, 64)]:
+        assert attn.decode_workspace_bytes(*shape) == expect(*shape)
+    assert attn.lib().attn_decode_workspace_bytes(1, 6, 2, 64, 64) == -1

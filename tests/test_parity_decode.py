@@ -1,0 +1,70 @@
+"""Decode against rolling caches (through the C ABI) against the fp64 oracle.
+
+Small problems cover every grouped-query ratio, head size, partially filled
+and wrapped caches, cache sizes that are not a multiple of the 64-slot tile,
+and mixed positions within a batch; the full-size workload (64 sequences at
+position 32767 against 4096-slot caches) is compared on every row.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_softmax_attention_04_b200 import synth
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def attn():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    import exact_softmax_attention_04_b200 as pkg
+    return pkg
+
+
+def _gpu(attn, q, kc, vc, pos, scale=None):
+    o, lse = attn.attn_decode(q.cuda(), kc.cuda(), vc.cuda(), torch.tensor(pos, dtype=torch.int32).cuda(),
+                              scale)
+    assert attn.sync_status() == attn.ATTN_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (8, 2), (8, 1)])
+@pytest.mark.parametrize("W", [1, 63, 64, 65, 200, 1024])
+def test_decode_small_in_full(attn, oracle_mod, d, H, Hkv, W):
+    B = 4
+    q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=W * 3 + H + d, q_std=2.0)
+    pos = [0, W // 2, W - 1, 3 * W + 7]  # one slot, half full, just full, wrapped
+    sc = 1.0 / np.sqrt(d)
+    o, lse = _gpu(attn, q, kc, vc, pos, sc)
+    o_ref, lse_ref = oracle_mod.attn_decode(q, kc, vc, pos, sc)
+    assert_close(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1),
+                 o_ref.reshape(-1, d), lse_ref.reshape(-1), f"W{W} H{H} Hkv{Hkv} d{d}")
+
+
+def test_decode_equals_forward_window_row(attn, oracle_mod):
+    """Caches filled from a sequence by the write rule: the decode of the last
+    position equals row T-1 of the forward pass with causal window W-1."""
+    B, H, Hkv, T, W, d = 2, 8, 2, 300, 128, 128
+    q, k, v = synth.make_qkv(B, H, T, d, seed=77, Hkv=Hkv)
+    kc, vc = synth.ring_from_sequence(k, W), synth.ring_from_sequence(v, W)
+    o_dec, l_dec = _gpu(attn, q[:, :, T - 1].contiguous(), kc, vc, [T - 1] * B)
+    o_fwd, l_fwd = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), None, True, W - 1)
+    assert attn.sync_status() == attn.ATTN_OK
+    assert (o_dec.float() - o_fwd[:, :, T - 1].float()).abs().max().item() <= 2e-2
+    assert (l_dec - l_fwd[:, :, T - 1]).abs().max().item() <= 1e-3
+
+
+def test_decode_full_size_workload_every_row(attn, oracle_mod):
+    wl = synth.DECODE_W4096
+    q, kc, vc = synth.make_decode(wl.B, wl.H, wl.Hkv, wl.W, wl.d, seed=wl.seed, q_std=wl.q_std)
+    o, lse = _gpu(attn, q, kc, vc, [wl.pos] * wl.B, wl.scale)
+    o_ref, lse_ref = oracle_mod.attn_decode(q, kc, vc, [wl.pos] * wl.B, wl.scale)
+    assert_close(o.float().cpu().numpy().reshape(-1, wl.d), lse.cpu().numpy().reshape(-1),
+                 o_ref.reshape(-1, wl.d), lse_ref.reshape(-1), wl.name)
+    o2, l2 = _gpu(attn, q, kc, vc, [wl.pos] * wl.B, wl.scale)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
