@@ -18,12 +18,16 @@ using namespace attn_host;
 
 bool g_dec_set[kMaxDevices][2][4] = {};
 
-// Splits of the W slots per (batch, kv head): enough CTAs to cover the SMs
-// a few times over, each split a whole number of 64-slot tiles.
+// Splits of the W slots per (batch, kv head): about ATTN_DECODE_CTAS_PER_SM
+// CTAs per SM of a 148-SM B200 in total, each split a whole number of
+// 64-slot tiles.
+#ifndef ATTN_DECODE_CTAS_PER_SM
+#define ATTN_DECODE_CTAS_PER_SM 4
+#endif
 void choose_splits(int64_t bkv, int W, int *nsplit, int *chunk)
 {
     const int tiles = (W + attn_sm100::DEC_TK - 1) / attn_sm100::DEC_TK;
-    const int64_t target = 4 * 148;
+    const int64_t target = ATTN_DECODE_CTAS_PER_SM * 148;
     int64_t ns = (target + bkv - 1) / bkv;
     if (ns < 1) ns = 1;
     if (ns > tiles) ns = tiles;
