@@ -58,6 +58,9 @@ def _load():
         lib.oracle_attn_bwd_rows_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
                                                  i64, vp, i64, vp, i64, vp, vp, vp]
         lib.oracle_attn_bwd_rows_f64.restype = ip
+        lib.oracle_attn_bwd_rows_gqa_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, i64, dbl, ip,
+                                                     i64, vp, i64, vp, i64, vp, vp, vp]
+        lib.oracle_attn_bwd_rows_gqa_f64.restype = ip
         lib.oracle_attn_decode_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp]
         lib.oracle_attn_decode_f64.restype = ip
         lib.oracle_num_threads.argtypes = []
@@ -177,6 +180,36 @@ def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=
                                       dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd_rows_f64 rejected its arguments (rc={rc})")
+    return dq, dk, dv
+
+
+def attn_bwd_rows_gqa(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=()
+                      ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Grouped-query backward for selected rows: q, dout [B, H, n, d], k, v
+    [B, Hkv, n, d] (all bf16 tensors or all fp64). dQ for flat query rows
+    (b*H + h)*n + i, dK and dV for flat key rows (b*Hkv + g)*n + j."""
+    lib = _load()
+    if q.shape != dout.shape or k.shape != v.shape or len(q.shape) != 4 or len(k.shape) != 4:
+        raise ValueError("q, dout must be [B, H, n, d] and k, v [B, Hkv, n, d]")
+    B, H, n, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape[0] != B or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k and v must be [B, Hkv, n, d]")
+    ins = [_bwd_input(x) for x in (q, k, v, dout)]
+    if len({t for _, t in ins}) != 1:
+        raise TypeError("q, k, v and dout must be all bf16 or all floating point")
+    qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64).reshape(-1))
+    kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64).reshape(-1))
+    dq = np.empty((qr.size, d), dtype=np.float64)
+    dk = np.empty((kr.size, d), dtype=np.float64)
+    dv = np.empty((kr.size, d), dtype=np.float64)
+    rc = lib.oracle_attn_bwd_rows_gqa_f64(ins[0][0].ctypes.data, ins[1][0].ctypes.data,
+                                          ins[2][0].ctypes.data, ins[3][0].ctypes.data, ins[0][1],
+                                          B, H, Hkv, n, d, float(scale), int(bool(causal)), int(window),
+                                          qr.ctypes.data, qr.size, kr.ctypes.data, kr.size,
+                                          dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd_rows_gqa_f64 rejected its arguments (rc={rc})")
     return dq, dk, dv
 
 

@@ -308,10 +308,11 @@ static double in_at(const void *p, int type, int64_t idx)
 }
 
 /* One query row's softmax statistics and, if dq != NULL, its gradient.
- * base = (b*H + h)*n*d is the head's offset; s and w are n-long scratch. */
+ * qbase = (b*H + h)*n*d is the query head's offset (q, dout), kbase that of
+ * its key/value head (k, v); s and dp are n-long scratch. */
 static void bwd_row(const void *q, const void *k, const void *v, const void *dout, int type,
-                    int64_t base, int64_t n, int64_t d, double scale, int causal, int64_t window,
-                    int64_t i, unsigned char *allowed, double *s, double *dp,
+                    int64_t qbase, int64_t kbase, int64_t n, int64_t d, double scale, int causal,
+                    int64_t window, int64_t i, unsigned char *allowed, double *s, double *dp,
                     double *lse_out, double *rowterm_out, double *dq)
 {
     oracle_mask_row(n, i, causal, window, allowed);
@@ -321,7 +322,7 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
             continue;
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c)
-            acc += in_at(q, type, base + i * d + c) * in_at(k, type, base + j * d + c);
+            acc += in_at(q, type, qbase + i * d + c) * in_at(k, type, kbase + j * d + c);
         s[j] = scale * acc;
         if (s[j] > M)
             M = s[j];
@@ -338,7 +339,7 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
             continue;
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c)
-            acc += in_at(dout, type, base + i * d + c) * in_at(v, type, base + j * d + c);
+            acc += in_at(dout, type, qbase + i * d + c) * in_at(v, type, kbase + j * d + c);
         dp[j] = acc;
         rowterm += exp(s[j] - lse) * acc;
     }
@@ -354,7 +355,7 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
                 continue;
             const double ds = exp(s[j] - lse) * (dp[j] - rowterm);
             for (int64_t c = 0; c < d; ++c)
-                dq[c] += ds * in_at(k, type, base + j * d + c);
+                dq[c] += ds * in_at(k, type, kbase + j * d + c);
         }
         for (int64_t c = 0; c < d; ++c)
             dq[c] *= scale;
@@ -362,33 +363,39 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
 }
 
 /*
- * Gradients for selected rows.
- *   q, k, v, dout : [B, H, n, d] inputs of element type `type`
+ * Gradients for selected rows, grouped-query form.
+ *   q, dout       : [B, H, n, d];  k, v : [B, Hkv, n, d], Hkv divides H; query
+ *                   head h of batch b reads key/value head b*Hkv + h/(H/Hkv)
+ *                   (element type `type`)
  *   qrows (nq)    : flat query rows (b*H + h)*n + i whose dQ is wanted -> dq (nq x d)
- *   krows (nk)    : flat key rows (b*H + h)*n + j whose dK, dV are wanted
- *                   -> dk, dv (nk x d each)
+ *   krows (nk)    : flat key rows (b*Hkv + g)*n + j whose dK, dV are wanted
+ *                   -> dk, dv (nk x d each). A key/value head's gradient sums
+ *                   the contributions of every query head that reads it.
  * Returns 0 on success, nonzero on bad input.
  */
-int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const void *dout, int type,
-                             int64_t B, int64_t H, int64_t n, int64_t d, double scale, int causal,
-                             int64_t window, const int64_t *qrows, int64_t nq, const int64_t *krows,
-                             int64_t nk, double *dq, double *dk, double *dv)
+int oracle_attn_bwd_rows_gqa_f64(const void *q, const void *k, const void *v, const void *dout, int type,
+                                 int64_t B, int64_t H, int64_t Hkv, int64_t n, int64_t d, double scale,
+                                 int causal, int64_t window, const int64_t *qrows, int64_t nq,
+                                 const int64_t *krows, int64_t nk, double *dq, double *dk, double *dv)
 {
-    if (!q || !k || !v || !dout || B <= 0 || H <= 0 || n <= 0 || d <= 0)
+    if (!q || !k || !v || !dout || B <= 0 || H <= 0 || Hkv <= 0 || n <= 0 || d <= 0)
+        return 1;
+    if (H % Hkv != 0)
         return 1;
     if (type != ORACLE_IN_BF16 && type != ORACLE_IN_F64)
         return 1;
     if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv)) || nq < 0 || nk < 0)
         return 1;
-    const int64_t rows_total = B * H * n;
+    const int64_t G = H / Hkv;
     for (int64_t r = 0; r < nq; ++r)
-        if (qrows[r] < 0 || qrows[r] >= rows_total)
+        if (qrows[r] < 0 || qrows[r] >= B * H * n)
             return 1;
     for (int64_t r = 0; r < nk; ++r)
-        if (krows[r] < 0 || krows[r] >= rows_total)
+        if (krows[r] < 0 || krows[r] >= B * Hkv * n)
             return 1;
 
-    /* heads that requested key rows belong to, and their per-row statistics */
+    /* query heads of the key/value heads with requested key rows, and their
+     * per-row statistics */
     const int64_t nheads = B * H;
     int64_t *slot = (int64_t *)malloc(sizeof(int64_t) * (size_t)nheads);
     if (!slot)
@@ -396,9 +403,13 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
     for (int64_t h = 0; h < nheads; ++h)
         slot[h] = -1;
     int64_t nstat = 0;
-    for (int64_t r = 0; r < nk; ++r)
-        if (slot[krows[r] / n] < 0)
-            slot[krows[r] / n] = nstat++;
+    for (int64_t r = 0; r < nk; ++r) {
+        const int64_t kvh = krows[r] / n;             /* b*Hkv + g */
+        const int64_t qh0 = (kvh / Hkv) * H + (kvh % Hkv) * G;
+        for (int64_t u = 0; u < G; ++u)
+            if (slot[qh0 + u] < 0)
+                slot[qh0 + u] = nstat++;
+    }
     int64_t *stat_head = (int64_t *)malloc(sizeof(int64_t) * (size_t)(nstat + 1));
     double *lse = (double *)malloc(sizeof(double) * (size_t)(nstat * n + 1));
     double *rowterm = (double *)malloc(sizeof(double) * (size_t)(nstat * n + 1));
@@ -423,44 +434,52 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
 #pragma omp atomic write
             bad = 1;
         } else {
-            /* 1. statistics of every row of the heads with requested key rows */
+            /* 1. statistics of every row of the query heads involved */
 #pragma omp for schedule(dynamic, 16)
             for (int64_t t = 0; t < nstat * n; ++t) {
                 const int64_t h = stat_head[t / n], i = t % n;
-                bwd_row(q, k, v, dout, type, h * n * d, n, d, scale, causal, window, i, allowed, s,
-                        dp, &lse[t], &rowterm[t], NULL);
+                const int64_t kvh = (h / H) * Hkv + (h % H) / G;
+                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, i,
+                        allowed, s, dp, &lse[t], &rowterm[t], NULL);
             }
             /* 2. dQ of the requested query rows */
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < nq; ++r) {
                 const int64_t h = qrows[r] / n, i = qrows[r] % n;
-                bwd_row(q, k, v, dout, type, h * n * d, n, d, scale, causal, window, i, allowed, s,
-                        dp, NULL, NULL, dq + r * d);
+                const int64_t kvh = (h / H) * Hkv + (h % H) / G;
+                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, i,
+                        allowed, s, dp, NULL, NULL, dq + r * d);
             }
-            /* 3. dK, dV of the requested key rows: sums over the queries that
-             * attend to key j, with each query's own LSE and row term */
+            /* 3. dK, dV of the requested key rows: sums over the query heads
+             * of the group and the queries that attend to key j, with each
+             * query's own LSE and row term */
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < nk; ++r) {
-                const int64_t h = krows[r] / n, j = krows[r] % n;
-                const int64_t base = h * n * d;
-                const double *L = lse + slot[h] * n;
-                const double *R = rowterm + slot[h] * n;
+                const int64_t kvh = krows[r] / n, j = krows[r] % n;
+                const int64_t kbase = kvh * n * d;
+                const int64_t qh0 = (kvh / Hkv) * H + (kvh % Hkv) * G;
                 double *gk = dk + r * d, *gv = dv + r * d;
                 for (int64_t c = 0; c < d; ++c)
                     gk[c] = gv[c] = 0.0;
-                for (int64_t i = 0; i < n; ++i) {
-                    if (!allowed_pair(i, j, causal, window))
-                        continue;
-                    double sij = 0.0, dpij = 0.0;
-                    for (int64_t c = 0; c < d; ++c) {
-                        sij += in_at(q, type, base + i * d + c) * in_at(k, type, base + j * d + c);
-                        dpij += in_at(dout, type, base + i * d + c) * in_at(v, type, base + j * d + c);
-                    }
-                    const double pij = exp(scale * sij - L[i]);
-                    const double dsij = pij * (dpij - R[i]);
-                    for (int64_t c = 0; c < d; ++c) {
-                        gv[c] += pij * in_at(dout, type, base + i * d + c);
-                        gk[c] += dsij * in_at(q, type, base + i * d + c);
+                for (int64_t u = 0; u < G; ++u) {
+                    const int64_t h = qh0 + u;
+                    const int64_t qbase = h * n * d;
+                    const double *L = lse + slot[h] * n;
+                    const double *R = rowterm + slot[h] * n;
+                    for (int64_t i = 0; i < n; ++i) {
+                        if (!allowed_pair(i, j, causal, window))
+                            continue;
+                        double sij = 0.0, dpij = 0.0;
+                        for (int64_t c = 0; c < d; ++c) {
+                            sij += in_at(q, type, qbase + i * d + c) * in_at(k, type, kbase + j * d + c);
+                            dpij += in_at(dout, type, qbase + i * d + c) * in_at(v, type, kbase + j * d + c);
+                        }
+                        const double pij = exp(scale * sij - L[i]);
+                        const double dsij = pij * (dpij - R[i]);
+                        for (int64_t c = 0; c < d; ++c) {
+                            gv[c] += pij * in_at(dout, type, qbase + i * d + c);
+                            gk[c] += dsij * in_at(q, type, qbase + i * d + c);
+                        }
                     }
                 }
                 for (int64_t c = 0; c < d; ++c)
@@ -476,6 +495,16 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
     free(lse);
     free(rowterm);
     return bad ? 2 : 0;
+}
+
+/* Multi-head form (Hkv = H); arguments as above. */
+int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const void *dout, int type,
+                             int64_t B, int64_t H, int64_t n, int64_t d, double scale, int causal,
+                             int64_t window, const int64_t *qrows, int64_t nq, const int64_t *krows,
+                             int64_t nk, double *dq, double *dk, double *dv)
+{
+    return oracle_attn_bwd_rows_gqa_f64(q, k, v, dout, type, B, H, H, n, d, scale, causal, window, qrows,
+                                        nq, krows, nk, dq, dk, dv);
 }
 
 /* ========================================================================

@@ -163,3 +163,48 @@ def test_bwd_oracle_rejects_bad_arguments(oracle_mod):
         oracle_mod.attn_bwd_rows(q, k, v[:, :, :4], do, 0.3, True, -1, [0], [])
     with pytest.raises(TypeError):
         oracle_mod.attn_bwd_rows(q, k, v, do.double(), 0.3, True, -1, [0], [])
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+def _textbook_gqa_forward(q, k, v, scale, causal, window):
+    """Grouped-query forward written with repeat_interleave: query head h
+    reads key/value head h // (H // Hkv)."""
+    H, Hkv = q.shape[1], k.shape[1]
+    idx = torch.arange(H) // (H // Hkv)
+    return _textbook_forward(q, k[:, idx], v[:, idx], scale, causal, window)
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 3), (4, 1)])
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 3), (False, 2)])
+def test_gqa_bwd_matches_autograd(oracle_mod, H, Hkv, causal, window):
+    """autograd through the repeat of K and V sums the group's gradients."""
+    B, n, d = 2, 13, 8
+    q, do = _rand((B, H, n, d), 61, 2.0), _rand((B, H, n, d), 62)
+    k, v = _rand((B, Hkv, n, d), 63), _rand((B, Hkv, n, d), 64)
+    qa, ka, va = (x.clone().requires_grad_(True) for x in (q, k, v))
+    (_textbook_gqa_forward(qa, ka, va, 0.4, causal, window) * do).sum().backward()
+    rows_q = np.arange(B * H * n)
+    rows_k = np.arange(B * Hkv * n)
+    dq, dk, dv = oracle_mod.attn_bwd_rows_gqa(q, k, v, do, 0.4, causal, window, rows_q, rows_k)
+    np.testing.assert_allclose(dq, qa.grad.numpy().reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, ka.grad.numpy().reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, va.grad.numpy().reshape(-1, d), rtol=0, atol=1e-12)
+
+
+def test_gqa_bwd_equals_group_sum_of_multi_head_gradients(oracle_mod):
+    """With K, V repeated per query head, multi-head dK, dV summed over each
+    group equal the grouped-query dK, dV; dQ is the same."""
+    B, H, Hkv, n, d = 1, 6, 2, 20, 8
+    q, k, v = synth.make_qkv(B, H, n, d, seed=65, Hkv=Hkv)
+    do = _rand(q.shape, 66).to(torch.bfloat16)
+    G = H // Hkv
+    kr, vr = k.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1)
+    dq_m, dk_m, dv_m = oracle_mod.attn_bwd(q, kr, vr, do, 0.3, True, 5)
+    rows_q, rows_k = np.arange(B * H * n), np.arange(B * Hkv * n)
+    dq_g, dk_g, dv_g = oracle_mod.attn_bwd_rows_gqa(q, k, v, do, 0.3, True, 5, rows_q, rows_k)
+    np.testing.assert_allclose(dq_g, dq_m.reshape(-1, d), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk_g.reshape(B, Hkv, n, d), dk_m.reshape(B, Hkv, G, n, d).sum(axis=2),
+                               rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv_g.reshape(B, Hkv, n, d), dv_m.reshape(B, Hkv, G, n, d).sum(axis=2),
+                               rtol=0, atol=1e-12)
