@@ -412,8 +412,6 @@ def run_bwd(args, wl, world, rank, local):
     import exact_softmax_attention_04_b200 as attn
     from exact_softmax_attention_04_b200 import synth
 
-    if wl.kv_heads != wl.H:
-        raise SystemExit("the backward pass takes K and V with H heads")
     dev = torch.device("cuda", local)
     q, k, v = synth.make_inputs(wl)
     do = synth.make_dout(wl.B, wl.H, wl.n, wl.d, seed=wl.seed)
@@ -495,12 +493,12 @@ def run_bwd(args, wl, world, rank, local):
         flops_per_row = flops / total
         probe = torch.randint(0, total, (16,), generator=g).numpy()
         t0 = time.perf_counter()
-        oracle.attn_bwd_rows(q, k, v, do, wl.scale, wl.causal, wl.window, probe, [])
+        oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, probe, [])
         dt = max(time.perf_counter() - t0, 1e-3)
         nrows = int(min(total, max(16, 16 * args.cpu_seconds / dt)))
         rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
         t0 = time.perf_counter()
-        dq_ref, _, _ = oracle.attn_bwd_rows(q, k, v, do, wl.scale, wl.causal, wl.window, rows, [])
+        dq_ref, _, _ = oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, rows, [])
         dt = time.perf_counter() - t0
         dq_gpu = grads[0].view(-1, wl.d)[torch.as_tensor(rows, device=dev)].float().cpu().numpy()
         diff = dq_gpu - dq_ref

@@ -29,7 +29,8 @@ ATTN_ERR_TOO_LARGE = 5
 # Every symbol include/attn.h declares.
 EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_release",
            "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
-           "attn_bwd", "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes")
+           "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes", "attn_decode",
+           "attn_decode_workspace_bytes")
 
 
 class AttnError(RuntimeError):
@@ -70,6 +71,9 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                              i, i, i, i, f, i, i, vp]
     lib.attn_bwd.restype = i
+    lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                 i, i, i, i, i, f, i, i, vp]
+    lib.attn_bwd_gqa.restype = i
     lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.attn_bwd_workspace_bytes.restype = i64
     lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, f, vp]
@@ -184,13 +188,16 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of the attention forward pass on the GPU.
 
-    q, k, v, o, dout: bf16 CUDA tensors [B, H, n, d], contiguous; o and lse
-    are attn_fwd's outputs for q, k, v with the same scale and mask; dout is
-    the upstream gradient dL/dO. ``workspace`` (optional) is a uint8 CUDA
-    tensor of at least bwd_workspace_bytes(B, H, n, d) bytes. Enqueued on
+    q, o, dout: bf16 CUDA tensors [B, H, n, d]; k, v: [B, H, n, d], or
+    [B, Hkv, n, d] with Hkv dividing H (grouped-query attention: dk, dv then
+    have Hkv heads and sum over each group). Contiguous; o and lse are
+    attn_fwd's outputs for q, k, v with the same scale and mask; dout is the
+    upstream gradient dL/dO. ``workspace`` (optional) is a uint8 CUDA tensor
+    of at least bwd_workspace_bytes(B, H, n, d) bytes. Enqueued on
     ``stream`` (default: the current stream).
     """
-    _check_qkv(q, k, v, device=True)
+    grouped = k.dim() == 4 and q.dim() == 4 and k.shape[1] != q.shape[1]
+    _check_qkv(q, k, v, device=True, grouped=grouped)
     for name, t in (("o", o), ("dout", dout)):
         if t.dtype != torch.bfloat16 or t.shape != q.shape or not t.is_contiguous() or \
                 t.device != q.device:
@@ -206,15 +213,15 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace.device != q.device or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous tensor on q's device")
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     with torch.cuda.device(q.device):
-        rc = lib().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                            B, H, n, d, float(scale), int(bool(causal)), int(window),
-                            _stream_handle(stream))
+        rc = lib().attn_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                B, H, k.shape[1], n, d, float(scale), int(bool(causal)), int(window),
+                                _stream_handle(stream))
     if rc != ATTN_OK:
-        raise AttnError(rc, "attn_bwd")
+        raise AttnError(rc, "attn_bwd_gqa")
     return dq, dk, dv
 
 

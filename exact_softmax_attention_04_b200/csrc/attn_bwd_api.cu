@@ -91,7 +91,7 @@ int prepare_kernel(Kernel kernel, int smem_bytes, uint32_t regs_launch)
 
 template <int D>
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-               const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int n,
+               const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int Hkv, int n,
                float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
 {
     using KV = attn_sm100::BwdKVCfg<D>;
@@ -99,11 +99,12 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     auto enc = encoder();
     if (!enc) return ATTN_ERR_CUDA;
     const int64_t bh = static_cast<int64_t>(B) * H;
+    const int64_t bhkv = static_cast<int64_t>(B) * Hkv;
     CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
-    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
-        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
-        !encode_bhnd(enc, &mdq, dq, bh, n, D) || !encode_bhnd(enc, &mdk, dk, bh, n, D) ||
-        !encode_bhnd(enc, &mdv, dv, bh, n, D))
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bhkv, n, D) ||
+        !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
+        !encode_bhnd(enc, &mdq, dq, bh, n, D) || !encode_bhnd(enc, &mdk, dk, bhkv, n, D) ||
+        !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -134,6 +135,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.lse2 = lse2;
     p.delta = delta;
     p.status = status;
+    p.heads = H;
+    p.kv_heads = Hkv;
     p.n = n;
     p.n_pad = n_pad;
     p.num_k_tiles = (n + attn_sm100::BN - 1) / attn_sm100::BN;
@@ -143,8 +146,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.causal = causal;
     p.window = effective_window(n, window);
 
-    // 2. dK, dV: one CTA per key tile
-    attn_sm100::attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bh * p.num_k_tiles), KV::THREADS,
+    // 2. dK, dV: one CTA per key tile of each key/value head
+    attn_sm100::attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bhkv * p.num_k_tiles), KV::THREADS,
                                           KV::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
@@ -158,17 +161,18 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 // kernel, accumulator -> bf16 dQ.
 template <int D>
 int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                     const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int n,
-                     float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+                     const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int Hkv,
+                     int n, float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
 {
     using Cfg = attn_sm100::FusedBwdCfg<D>;
     auto enc = encoder();
     if (!enc) return ATTN_ERR_CUDA;
     const int64_t bh = static_cast<int64_t>(B) * H;
+    const int64_t bhkv = static_cast<int64_t>(B) * Hkv;
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
-    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bh, n, D) ||
-        !encode_bhnd(enc, &mv, v, bh, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
-        !encode_bhnd(enc, &mdk, dk, bh, n, D) || !encode_bhnd(enc, &mdv, dv, bh, n, D))
+    if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bhkv, n, D) ||
+        !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
+        !encode_bhnd(enc, &mdk, dk, bhkv, n, D) || !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
     {
         std::lock_guard<std::mutex> lk(g_mu);
@@ -199,6 +203,8 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
     p.lse2 = lse2;
     p.delta = delta;
     p.status = status;
+    p.heads = H;
+    p.kv_heads = Hkv;
     p.n = n;
     p.n_pad = n_pad;
     p.num_k_tiles = (n + attn_sm100::BN - 1) / attn_sm100::BN;
@@ -206,7 +212,7 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
     p.window = effective_window(n, window);
-    const unsigned grid = static_cast<unsigned>(bh * p.num_k_tiles);
+    const unsigned grid = static_cast<unsigned>(bhkv * p.num_k_tiles);
     attn_sm100::attn_bwd_fused_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
                                                                                           mdv, macc, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -227,12 +233,14 @@ extern "C" int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d)
     return static_cast<int64_t>(workspace_layout(static_cast<int64_t>(B) * H, n, d).total);
 }
 
-extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
-                        const void *dout, void *dq, void *dk, void *dv, void *workspace,
-                        size_t workspace_bytes, int B, int H, int n, int d, float scale, int causal,
-                        int window, void *stream)
+namespace {
+
+int bwd_entry(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+              void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int Hkv,
+              int n, int d, float scale, int causal, int window, void *stream)
 {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
+    if (Hkv <= 0 || H <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
     const int rc = check_bwd_args(B, H, n, d, scale, causal);
     if (rc != ATTN_OK) return rc;
     for (const void *ptr : {q, k, v, o, dout, static_cast<const void *>(dq), static_cast<const void *>(dk),
@@ -247,8 +255,28 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
     if (fused_for(d))
-        return launch_bwd_fused<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window,
+        return launch_bwd_fused<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, Hkv, n, scale, causal, window,
                                     st, dev, status);
-    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, n, scale, causal, window, st, dev,
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, Hkv, n, scale, causal, window, st, dev,
                            status);
+}
+
+}  // namespace
+
+extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                        const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                        size_t workspace_bytes, int B, int H, int n, int d, float scale, int causal,
+                        int window, void *stream)
+{
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, n, d, scale, causal,
+                     window, stream);
+}
+
+extern "C" int attn_bwd_gqa(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                            const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                            size_t workspace_bytes, int B, int H, int Hkv, int n, int d, float scale, int causal,
+                            int window, void *stream)
+{
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, n, d, scale,
+                     causal, window, stream);
 }

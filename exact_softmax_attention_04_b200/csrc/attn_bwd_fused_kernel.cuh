@@ -7,7 +7,8 @@
 //
 // The gradients, the recompute and the roles are those described in
 // attn_bwd_kernel.cuh; this file differs in:
-//   2. attn_bwd_fused_kernel: one CTA per (batch*head, 128-key tile). Per
+//   2. attn_bwd_fused_kernel: one CTA per (batch * key/value head, 128-key
+//      tile), walking the query tiles of every query head of the group. Per
 //      query tile it runs five tcgen05 MMAs:
 //        S^T  = K_j Q_i^T        (smem x smem -> TMEM, 128 keys x 128 queries)
 //        dP^T = V_j dO_i^T       (smem x smem -> TMEM)
@@ -46,6 +47,8 @@ struct FusedBwdParams {
     const float *lse2;   // [B*H, n_pad] LSE * log2(e)
     const float *delta;  // [B*H, n_pad] dO . O
     int *status;
+    int heads;           // H: query heads per batch
+    int kv_heads;        // H_kv: key/value heads per batch (divides H)
     int n;
     int n_pad;           // n rounded up to a multiple of 128
     int num_k_tiles;     // ceil(n / 128)
@@ -223,13 +226,22 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
 
     // Work: the key tiles of one head are adjacent in blockIdx (Q / dO reuse
     // in L2); under a causal mask the early key tiles (most query tiles) first.
-    const int bh = blockIdx.x / p.num_k_tiles;
+    // The CTA walks the query tiles [qlo, qhi) of every query head reading
+    // this key/value head (grouped-query attention; one head for multi-head
+    // attention): item it is query tile qlo + it % nq of the group's head
+    // it / nq.
+    const int bkv = blockIdx.x / p.num_k_tiles;
+    const int G = p.heads / p.kv_heads;
+    const int bh0 = (bkv / p.kv_heads) * p.heads + (bkv % p.kv_heads) * G;
     const int kt = static_cast<int>(blockIdx.x % p.num_k_tiles);
     const int k0 = kt * BN;
     const int n = p.n;
     int qlo, qhi;
     query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
     const int nq = qhi - qlo;  // >= 1: query k0 attends to key k0
+    const int nitems = G * nq;
+    auto item_q0 = [&](int it) { return (qlo + it % nq) * BM; };
+    auto item_bh = [&](int it) { return bh0 + it / nq; };
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -274,15 +286,16 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
         mbar_arrive_expect_tx_if(leader, kv_full, 2 * C::TILE_BYTES);
 #pragma unroll
         for (int b = 0; b < C::BOXES; ++b) {
-            tma_load_3d_if(leader, sK + b * BOX_BYTES, &tmK, kv_full, b * BOX_COLS, k0, bh);
-            tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bh);
+            tma_load_3d_if(leader, sK + b * BOX_BYTES, &tmK, kv_full, b * BOX_COLS, k0, bkv);
+            tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bkv);
         }
         int issued = 0;
-        for (int it = 0; it < nq; ++it) {
+        for (int it = 0; it < nitems; ++it) {
             const int s = it % NST;
             if (it >= NST && !__all_sync(0xffffffffu, wt.wait(q_empty(s), ((it / NST) & 1u) ^ 1u)))
                 break;
-            const int q0 = (qlo + it) * BM;
+            const int q0 = item_q0(it);
+            const int bh = item_bh(it);
 #ifdef ATTN_FAULT_BWD_DROP_FIRST_Q
             // Test hook (never defined in the library build): the first Q/dO
             // stage is never loaded, so the MMA warp's wait on it must expire
@@ -356,7 +369,7 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
             issue_s(0);
             issue_dp(0);
         }
-        for (int it = 0; ok && it < nq; ++it) {
+        for (int it = 0; ok && it < nitems; ++it) {
             const int s = it % NST;
             const uint64_t q_mn = smem_desc_sw128(sQ(s), BOX_BYTES, 1024);
             const uint64_t do_mn = smem_desc_sw128(sdO(s), BOX_BYTES, 1024);
@@ -370,7 +383,7 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
                                do_mn + static_cast<uint64_t>(kk * 128), idesc_acc,
                                (it > 0 || kk > 0) ? 1u : 0u);
             }
-            if (it + 1 < nq) {
+            if (it + 1 < nitems) {
                 if (!(ok = wait(q_full((it + 1) % NST), ((it + 1) / NST) & 1u))) break;
                 issue_s(it + 1);
             }
@@ -391,7 +404,7 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
             mma_commit_if(leader, dq_full);
             mma_commit_if(leader, ds_free);
             mma_commit_if(leader, q_empty(s));
-            if (it + 1 < nq) {
+            if (it + 1 < nitems) {
                 // with D = 128, dQ_it sits in dP's columns: the drain must have read it
                 if (D == 128 && !(ok = wait(dq_free, it & 1u))) break;
                 issue_dp(it + 1);
@@ -422,12 +435,12 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
                              f2u(u2f(v[4 * j + 2]) * sc), f2u(u2f(v[4 * j + 3]) * sc));
             }
         };
-        for (int it = 0; it < nq; ++it) {
+        for (int it = 0; it < nitems; ++it) {
             // all four warps take the same decision (they meet at named
             // barriers below)
             if (!named_bar_and(3, BM, wt.wait(dq_full, it & 1u))) break;
             tc_fence_after();
-            const int q0 = (qlo + it) * BM;
+            const int q0 = item_q0(it);
 #pragma unroll 1
             for (int hf = 0; hf < D / 64; ++hf) {
                 uint32_t va[32], vb[32];
@@ -446,8 +459,8 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
                 fence_proxy_async_smem();
                 named_bar_sync(3, BM);
                 if (issuer) {
-                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, bh);
-                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, bh);
+                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, item_bh(it));
+                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, item_bh(it));
                     tma_store_commit();
                 }
             }
@@ -469,9 +482,9 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
         bool ok = true;
-        for (int it = 0; it < nq; ++it) {
+        for (int it = 0; it < nitems; ++it) {
             const int s = it % NST;
-            const int q0 = (qlo + it) * BM;
+            const int q0 = item_q0(it);
             ok = __all_sync(0xffffffffu, wt.wait(s_full, it & 1u));
             if (!ok) break;
             tc_fence_after();
@@ -597,7 +610,7 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
             named_bar_sync(1 + h, BN);
             if (r == 0) {
                 const CUtensorMap *map = h ? &tmdK : &tmdV;
-                for (int b = 0; b < C::BOXES; ++b) tma_store_3d(map, stage + b * BOX_BYTES, b * BOX_COLS, k0, bh);
+                for (int b = 0; b < C::BOXES; ++b) tma_store_3d(map, stage + b * BOX_BYTES, b * BOX_COLS, k0, bkv);
                 tma_store_commit();
                 tma_store_wait_read0();
             }

@@ -14,17 +14,21 @@
 // Three launches on one stream:
 //   1. attn_bwd_prep_kernel: delta_i and LSE_i * log2(e) per row, padded to a
 //      whole number of 128-row tiles per head.
-//   2. attn_bwd_dkdv_kernel: one CTA per (batch*head, 128-key tile j). K_j,
-//      V_j stay in shared memory; the CTA walks the query tiles i that attend
-//      to tile j and runs, per query tile, four tcgen05 MMAs:
+//   2. attn_bwd_dkdv_kernel: one CTA per (batch * key/value head, 128-key
+//      tile j). K_j, V_j stay in shared memory; the CTA walks the query tiles
+//      i that attend to tile j, for every query head that reads this
+//      key/value head (one for multi-head attention, H / H_kv for
+//      grouped-query attention, whose dK and dV sum over the group), and
+//      runs, per query tile, four tcgen05 MMAs:
 //        S^T  = K_j Q_i^T   (smem x smem -> TMEM, 128 keys x 128 queries)
 //        dP^T = V_j dO_i^T  (smem x smem -> TMEM)
 //        dV  += P^T dO_i    (P^T in TMEM, over S^T's columns)
 //        dK  += dS^T Q_i    (dS^T in TMEM, over dP^T's columns)
 //      dV and dK accumulate in TMEM over the walk and are stored once.
-//   3. attn_bwd_dq_kernel: one CTA per (batch*head, 128-query tile i), Q_i
-//      and dO_i held in TMEM as MMA operands; it walks the key tiles j that
-//      tile i attends to and runs three MMAs per key tile:
+//   3. attn_bwd_dq_kernel: one CTA per (batch * query head, 128-query tile
+//      i), Q_i and dO_i held in TMEM as MMA operands; it walks the key tiles j
+//      of the head's key/value head that tile i attends to and runs three MMAs
+//      per key tile:
 //        S  = Q_i K_j^T, dP = dO_i V_j^T   (TMEM x smem -> TMEM)
 //        dQ += dS K_j                      (dS in TMEM, over dP's columns)
 //      dQ accumulates in TMEM and is stored once.
@@ -64,6 +68,8 @@ struct BwdParams {
     const float *lse2;   // [B*H, n_pad] LSE * log2(e)
     const float *delta;  // [B*H, n_pad] dO . O
     int *status;
+    int heads;           // H: query heads per batch
+    int kv_heads;        // H_kv: key/value heads per batch (divides H)
     int n;
     int n_pad;           // n rounded up to a multiple of 128
     int num_k_tiles;     // ceil(n / 128)
@@ -282,15 +288,24 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
 
     const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0);
 
-    // Work: the key tiles of one head are adjacent in blockIdx (Q / dO reuse
-    // in L2); under a causal mask the early key tiles (most query tiles) first.
-    const int bh = blockIdx.x / p.num_k_tiles;
+    // Work: the key tiles of one key/value head are adjacent in blockIdx (Q /
+    // dO reuse in L2); under a causal mask the early key tiles (most query
+    // tiles) first. The CTA walks the query tiles [qlo, qhi) of every query
+    // head of the group (grouped-query attention: G = H / H_kv heads share
+    // this key/value head; G = 1 for multi-head attention), item it being
+    // query tile qlo + it % nq of the group's head it / nq.
+    const int bkv = blockIdx.x / p.num_k_tiles;
     const int kt = static_cast<int>(blockIdx.x % p.num_k_tiles);
     const int k0 = kt * BN;
     const int n = p.n;
+    const int G = p.heads / p.kv_heads;
+    const int bh0 = (bkv / p.kv_heads) * p.heads + (bkv % p.kv_heads) * G;  // first query head
     int qlo, qhi;
     query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
     const int nq = qhi - qlo;  // >= 1: query k0 attends to key k0
+    const int nitems = G * nq;
+    auto item_q0 = [&](int it) { return (qlo + it % nq) * BM; };
+    auto item_bh = [&](int it) { return bh0 + it / nq; };
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -331,15 +346,16 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
         mbar_arrive_expect_tx_if(leader, kv_full, 2 * C::TILE_BYTES);
 #pragma unroll
         for (int b = 0; b < C::BOXES; ++b) {
-            tma_load_3d_if(leader, sK + b * BOX_BYTES, &tmK, kv_full, b * BOX_COLS, k0, bh);
-            tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bh);
+            tma_load_3d_if(leader, sK + b * BOX_BYTES, &tmK, kv_full, b * BOX_COLS, k0, bkv);
+            tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bkv);
         }
         int issued = 0;
-        for (int it = 0; it < nq; ++it) {
+        for (int it = 0; it < nitems; ++it) {
             const int s = it % NST;
             if (it >= NST && !__all_sync(0xffffffffu, wt.wait(q_empty(s), ((it / NST) & 1u) ^ 1u)))
                 break;
-            const int q0 = (qlo + it) * BM;
+            const int q0 = item_q0(it);
+            const int bh = item_bh(it);
 #ifdef ATTN_FAULT_BWD_DROP_FIRST_Q
             // Test hook (never defined in the library build): the first Q/dO
             // stage is never loaded, so the MMA warp's wait on it must expire
@@ -409,7 +425,7 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             issue_s(0);
             issue_dp(0);
         }
-        for (int it = 0; ok && it < nq; ++it) {
+        for (int it = 0; ok && it < nitems; ++it) {
             const int s = it % NST;
             const uint64_t q_mn = smem_desc_sw128(sQ(s), BOX_BYTES, 1024);
             const uint64_t do_mn = smem_desc_sw128(sdO(s), BOX_BYTES, 1024);
@@ -423,7 +439,7 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
                                do_mn + static_cast<uint64_t>(kk * 128), idesc_acc,
                                (it > 0 || kk > 0) ? 1u : 0u);
             }
-            if (it + 1 < nq) {
+            if (it + 1 < nitems) {
                 if (!(ok = wait(q_full((it + 1) % NST), ((it + 1) / NST) & 1u))) break;
                 issue_s(it + 1);
             }
@@ -437,7 +453,7 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
                                (it > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit_if(leader, q_empty(s));
-            if (it + 1 < nq) issue_dp(it + 1);
+            if (it + 1 < nitems) issue_dp(it + 1);
         }
         if (ok) mma_commit_if(leader, kv_done);
         // Every MMA this warp issued must finish before TMEM is freed.
@@ -454,9 +470,9 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
         bool ok = true;
-        for (int it = 0; it < nq; ++it) {
+        for (int it = 0; it < nitems; ++it) {
             const int s = it % NST;
-            const int q0 = (qlo + it) * BM;
+            const int q0 = item_q0(it);
             ok = __all_sync(0xffffffffu, wt.wait(s_full, it & 1u));
             if (!ok) break;
             tc_fence_after();
@@ -559,7 +575,7 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             named_bar_sync(1 + h, BN);
             if (r == 0) {
                 const CUtensorMap *map = h ? &tmdK : &tmdV;
-                for (int b = 0; b < C::BOXES; ++b) tma_store_3d(map, stage + b * BOX_BYTES, b * BOX_COLS, k0, bh);
+                for (int b = 0; b < C::BOXES; ++b) tma_store_3d(map, stage + b * BOX_BYTES, b * BOX_COLS, k0, bkv);
                 tma_store_commit();
                 tma_store_wait_read0();
             }
@@ -610,6 +626,8 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     // within a head the late tiles (the most key tiles under a causal mask)
     // first.
     const int bh = blockIdx.x / p.num_q_tiles;
+    // key/value head of this query head (grouped-query attention)
+    const int bkv = (bh / p.heads) * p.kv_heads + (bh % p.heads) / (p.heads / p.kv_heads);
     const int qt = p.num_q_tiles - 1 - static_cast<int>(blockIdx.x % p.num_q_tiles);
     const int q0 = qt * BM;
     const int n = p.n;
@@ -673,7 +691,7 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             const int k0 = (jlo + i / 2) * BN;
 #pragma unroll
             for (int b = 0; b < C::BOXES; ++b)
-                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bh);
+                tma_load_3d_if(leader, sKV(slot) + b * BOX_BYTES, map, kv_full(slot), b * BOX_COLS, k0, bkv);
             ++issued;
         }
         wt.drain(qd_full, 0);

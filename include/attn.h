@@ -213,8 +213,27 @@ ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o
                       void *workspace, size_t workspace_bytes, int B, int H, int n, int d,
                       float scale, int causal, int window, void *stream);
 
-/* Device workspace bytes attn_bwd needs for this shape, or -1 if the shape
- * is invalid or unsupported. */
+/*
+ * attn_bwd_gqa - the backward pass of attn_fwd_gqa (grouped-query and
+ * multi-query attention): K, V, dK and dV have Hkv heads, Hkv divides H,
+ * query head h reads key/value head h / (H / Hkv), and the gradient of a
+ * key/value head sums the contributions of every query head that reads it.
+ *
+ *   q, o, dout, dq : device, bf16 [B, H, n, d]
+ *   k, v, dk, dv   : device, bf16 [B, Hkv, n, d]
+ *   lse            : device, fp32 [B, H, n]
+ *   workspace      : at least attn_bwd_workspace_bytes(B, H, n, d) bytes
+ * Everything else as attn_bwd; Hkv < 1 or not dividing H gives
+ * ATTN_ERR_INVALID.
+ */
+ATTN_API int attn_bwd_gqa(const void *q, const void *k, const void *v, const void *o,
+                          const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                          void *workspace, size_t workspace_bytes, int B, int H, int Hkv, int n,
+                          int d, float scale, int causal, int window, void *stream);
+
+/* Device workspace bytes attn_bwd (and attn_bwd_gqa, with the query head
+ * count H) needs for this shape, or -1 if the shape is invalid or
+ * unsupported. */
 ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
 
 /*

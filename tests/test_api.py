@@ -197,3 +197,11 @@ def test_decode_workspace_size(attn):
     for shape in [(1, 1, 1, 1, 64), (2, 8, 2, 4096, 128), (64, 32, 8, 4096, 128), (3, 4, 4, 200, 64)]:
         assert attn.decode_workspace_bytes(*shape) == expect(*shape)
     assert attn.lib().attn_decode_workspace_bytes(1, 6, 2, 64, 64) == -1
+
+
+def test_bwd_gqa_entry_point_rejects_bad_head_counts(attn):
+    lib = attn.lib()
+    for Hkv in (0, -2, 3, 16):
+        rc = lib.attn_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40,
+                              1, 8, Hkv, 128, 64, 0.125, 1, -1, None)
+        assert rc == attn.ATTN_ERR_INVALID, Hkv

@@ -129,3 +129,40 @@ def test_bwd_full_size_workloads_sampled(attn, oracle_mod, wl):
                        [dq_ref, dk_ref, dv_ref], wl.name)
     for g in grads:
         assert bool(torch.isfinite(g.float()).all())
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 3), (8, 1)])
+@pytest.mark.parametrize("causal,window", [(False, -1), (True, -1), (True, 100), (False, 60)])
+def test_gqa_bwd_small_in_full(attn, oracle_mod, d, H, Hkv, causal, window):
+    B, n = 2, 300
+    q, k, v = synth.make_qkv(B, H, n, d, seed=H * 10 + Hkv + d, q_std=2.0, Hkv=Hkv)
+    do = synth.make_dout(B, H, n, d, seed=H * 10 + Hkv + d)
+    sc = 1.0 / np.sqrt(d)
+    grads = _fwd_bwd(attn, q, k, v, do, causal, window, sc)
+    rows_q, rows_k = np.arange(B * H * n), np.arange(B * Hkv * n)
+    refs = oracle_mod.attn_bwd_rows_gqa(q, k, v, do, sc, causal, window, rows_q, rows_k)
+    assert_grads_close([g.float().cpu().numpy().reshape(-1, d) for g in grads], refs,
+                       f"gqa H{H} Hkv{Hkv} d{d} c{causal} w{window}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa_bwd_equals_group_sums_of_multi_head(attn, d):
+    """Grouped-query dK, dV equal the group sums of the multi-head gradients
+    on repeated K/V (each rounded to bf16 separately, hence a tolerance);
+    dQ is the same computation."""
+    B, H, Hkv, n = 1, 8, 2, 500
+    q, k, v = synth.make_qkv(B, H, n, d, seed=80 + d, Hkv=Hkv)
+    do = synth.make_dout(B, H, n, d, seed=80 + d)
+    g = _fwd_bwd(attn, q, k, v, do, True, -1)
+    G = H // Hkv
+    m = _fwd_bwd(attn, q, k.repeat_interleave(G, dim=1), v.repeat_interleave(G, dim=1), do, True, -1)
+    if d == 128:
+        assert torch.equal(g[0], m[0])  # the dQ kernel does the same work in the same order
+    else:
+        assert (g[0].float() - m[0].float()).abs().max().item() <= 1e-2 * m[0].float().abs().max().item()
+    for a, b in ((g[1], m[1]), (g[2], m[2])):
+        ref = b.float().view(B, Hkv, G, n, d).sum(dim=2)
+        assert (a.float() - ref).abs().max().item() <= 2e-2 * ref.abs().max().item()
