@@ -168,13 +168,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest x over all ranks (every rank gets it); the timed interval
+    of a multi-GPU run is the slowest rank's."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job throughput of independent replicas: every rank processes
+    units_per_rank per step, the job takes the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
 
 
 def cpu_baseline_leg(wl, o_gpu=None, lse_gpu=None, target_s: float = 15.0):
@@ -235,7 +243,7 @@ def run_reference(args, wl, world, rank):
     t0 = time.perf_counter()
     oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe)
     per_row = max((time.perf_counter() - t0) / 32, 1e-6)
-    budget = 120.0 / max(1, args.steps + args.warmup)
+    budget = args.reference_seconds / max(1, args.steps + args.warmup)
     nrows = int(max(8, min(total, budget / per_row)))
     samples = [np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
                for _ in range(args.steps + args.warmup)]
@@ -338,7 +346,7 @@ def run_ours(args, wl, world, rank, local):
     total_ms = max_over_ranks(start_all.elapsed_time(end_all), world)
     per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value = replica_throughput(flops, args.steps, total_ms, world) / 1e12
 
     bf16_peak, hbm_peak, peak_src = peaks()
     achieved = flops / (per_launch_ms / 1e3) / 1e12
@@ -466,7 +474,7 @@ def run_bwd(args, wl, world, rank, local):
         return 0
     bf16_peak, _, peak_src = peaks()
     line = {
-        "metric": BWD_METRIC, "value": world * flops * args.steps / (total_ms / 1e3) / 1e12,
+        "metric": BWD_METRIC, "value": replica_throughput(flops, args.steps, total_ms, world) / 1e12,
         "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -663,6 +671,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="B8-H8-n8192-d64-none")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="oracle work budget of the --impl reference arm (warm-up and timed steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every target workload (kernel only, median of --steps, L2 flushed)")
