@@ -90,6 +90,19 @@ def attended_pairs_per_head(n: int, causal: bool, window: int) -> int:
     return n * n
 
 
+def attended_pairs_block(n: int, block: int, causal: bool) -> int:
+    """Pairs of the block-local mask in one head: query i attends to the keys
+    of its own block floor(i/b) and of the previous block (j <= i as well
+    when causal)."""
+    total = 0
+    for i in range(n):
+        bi = i // block
+        lo = max(0, (bi - 1) * block)
+        hi = i if causal else min(n - 1, (bi + 1) * block - 1)
+        total += hi - lo + 1
+    return total
+
+
 def unmasked_flops(wl: "Workload") -> int:
     """4*d FLOPs per attended pair (2*d for QK^T, 2*d for PV), times B*H."""
     return 4 * wl.d * attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H

@@ -43,23 +43,23 @@ def _load():
         build()
         lib = ctypes.CDLL(_LIB)
         i64, dbl, vp, ip = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
-        lib.oracle_attn_rows_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, ip,
+        lib.oracle_attn_rows_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, i64, ip,
                                              vp, i64, vp, vp, vp]
         lib.oracle_attn_rows_f64.restype = ip
         lib.oracle_attn_rows_gqa_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, dbl, ip, i64,
-                                                 ip, vp, i64, vp, vp, vp]
+                                                 i64, ip, vp, i64, vp, vp, vp]
         lib.oracle_attn_rows_gqa_f64.restype = ip
-        lib.oracle_attn_fwd_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, vp, vp]
+        lib.oracle_attn_fwd_f64.argtypes = [vp, vp, vp, i64, i64, i64, i64, dbl, ip, i64, i64, vp, vp]
         lib.oracle_attn_fwd_f64.restype = ip
         lib.oracle_matmul_f64.argtypes = [i64, i64, i64, vp, ip, vp, ip, vp]
         lib.oracle_matmul_f64.restype = ip
-        lib.oracle_mask_row.argtypes = [i64, i64, ip, i64, vp]
+        lib.oracle_mask_row.argtypes = [i64, i64, ip, i64, i64, vp]
         lib.oracle_mask_row.restype = ip
         lib.oracle_attn_bwd_rows_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
-                                                 i64, vp, i64, vp, i64, vp, vp, vp]
+                                                 i64, i64, vp, i64, vp, i64, vp, vp, vp]
         lib.oracle_attn_bwd_rows_f64.restype = ip
         lib.oracle_attn_bwd_rows_gqa_f64.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, i64, dbl, ip,
-                                                     i64, vp, i64, vp, i64, vp, vp, vp]
+                                                     i64, i64, vp, i64, vp, i64, vp, vp, vp]
         lib.oracle_attn_bwd_rows_gqa_f64.restype = ip
         lib.oracle_attn_decode_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp]
         lib.oracle_attn_decode_f64.restype = ip
@@ -78,9 +78,11 @@ def _bits(t) -> np.ndarray:
 
 
 def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
-              kernel: int = KERNEL_SOFTMAX, want_weights: bool = False
+              kernel: int = KERNEL_SOFTMAX, want_weights: bool = False, block: int = 0
               ) -> Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]:
-    """O (nrows x d), LSE (nrows) and optionally weights (nrows x n) for flat rows."""
+    """O (nrows x d), LSE (nrows) and optionally weights (nrows x n) for flat
+    rows. block > 0 selects the block-local mask (own block and the previous
+    one; window must then be < 0)."""
     lib = _load()
     if not (q.shape == k.shape == v.shape) or len(q.shape) != 4:
         raise ValueError("q, k and v must all be [B, H, n, d] (see attn_rows_gqa for fewer K/V heads)")
@@ -91,7 +93,7 @@ def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
     lse = np.empty(rows.size, dtype=np.float64)
     w = np.empty((rows.size, n), dtype=np.float64) if want_weights else None
     rc = lib.oracle_attn_rows_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, n, d,
-                                  float(scale), int(bool(causal)), int(window), int(kernel),
+                                  float(scale), int(bool(causal)), int(window), int(block), int(kernel),
                                   rows.ctypes.data, rows.size, o.ctypes.data, lse.ctypes.data,
                                   w.ctypes.data if w is not None else None)
     if rc != 0:
@@ -100,7 +102,7 @@ def attn_rows(q, k, v, scale: float, causal: bool, window: int, rows,
 
 
 def attn_rows_gqa(q, k, v, scale: float, causal: bool, window: int, rows,
-                  kernel: int = KERNEL_SOFTMAX) -> Tuple[np.ndarray, np.ndarray]:
+                  kernel: int = KERNEL_SOFTMAX, block: int = 0) -> Tuple[np.ndarray, np.ndarray]:
     """Grouped-query form: q [B, H, n, d], k and v [B, Hkv, n, d], Hkv | H.
     O (nrows x d) and LSE (nrows) for flat query rows (b*H + h)*n + i."""
     lib = _load()
@@ -113,14 +115,14 @@ def attn_rows_gqa(q, k, v, scale: float, causal: bool, window: int, rows,
     o = np.empty((rows.size, d), dtype=np.float64)
     lse = np.empty(rows.size, dtype=np.float64)
     rc = lib.oracle_attn_rows_gqa_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, Hkv, n, d,
-                                      float(scale), int(bool(causal)), int(window), int(kernel),
+                                      float(scale), int(bool(causal)), int(window), int(block), int(kernel),
                                       rows.ctypes.data, rows.size, o.ctypes.data, lse.ctypes.data, None)
     if rc != 0:
         raise ValueError(f"oracle_attn_rows_gqa_f64 rejected its arguments (rc={rc})")
     return o, lse
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1
+def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1, block: int = 0
              ) -> Tuple[np.ndarray, np.ndarray]:
     """Full O [B,H,n,d] and LSE [B,H,n] in fp64."""
     lib = _load()
@@ -131,7 +133,7 @@ def attn_fwd(q, k, v, scale: float, causal: bool, window: int = -1
     o = np.empty((B, H, n, d), dtype=np.float64)
     lse = np.empty((B, H, n), dtype=np.float64)
     rc = lib.oracle_attn_fwd_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, B, H, n, d,
-                                 float(scale), int(bool(causal)), int(window),
+                                 float(scale), int(bool(causal)), int(window), int(block),
                                  o.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd_f64 rejected its arguments (rc={rc})")
@@ -153,8 +155,8 @@ def _bwd_input(t):
     return np.ascontiguousarray(np.asarray(t, dtype=np.float64)), IN_F64
 
 
-def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=()
-                  ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=(),
+                  block: int = 0) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Backward pass for selected rows. q, k, v, dout: [B, H, n, d], all bf16
     torch tensors or all fp64 arrays. Returns dQ for the flat query rows
     ``qrows`` (len x d) and dK, dV for the flat key rows ``krows`` (len x d
@@ -175,7 +177,7 @@ def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=
     dv = np.empty((kr.size, d), dtype=np.float64)
     rc = lib.oracle_attn_bwd_rows_f64(ins[0][0].ctypes.data, ins[1][0].ctypes.data,
                                       ins[2][0].ctypes.data, ins[3][0].ctypes.data, typ,
-                                      B, H, n, d, float(scale), int(bool(causal)), int(window),
+                                      B, H, n, d, float(scale), int(bool(causal)), int(window), int(block),
                                       qr.ctypes.data, qr.size, kr.ctypes.data, kr.size,
                                       dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
     if rc != 0:
@@ -183,8 +185,8 @@ def attn_bwd_rows(q, k, v, dout, scale: float, causal: bool, window: int, qrows=
     return dq, dk, dv
 
 
-def attn_bwd_rows_gqa(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=()
-                      ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+def attn_bwd_rows_gqa(q, k, v, dout, scale: float, causal: bool, window: int, qrows=(), krows=(),
+                      block: int = 0) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Grouped-query backward for selected rows: q, dout [B, H, n, d], k, v
     [B, Hkv, n, d] (all bf16 tensors or all fp64). dQ for flat query rows
     (b*H + h)*n + i, dK and dV for flat key rows (b*Hkv + g)*n + j."""
@@ -206,19 +208,19 @@ def attn_bwd_rows_gqa(q, k, v, dout, scale: float, causal: bool, window: int, qr
     rc = lib.oracle_attn_bwd_rows_gqa_f64(ins[0][0].ctypes.data, ins[1][0].ctypes.data,
                                           ins[2][0].ctypes.data, ins[3][0].ctypes.data, ins[0][1],
                                           B, H, Hkv, n, d, float(scale), int(bool(causal)), int(window),
-                                          qr.ctypes.data, qr.size, kr.ctypes.data, kr.size,
+                                          int(block), qr.ctypes.data, qr.size, kr.ctypes.data, kr.size,
                                           dq.ctypes.data, dk.ctypes.data, dv.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd_rows_gqa_f64 rejected its arguments (rc={rc})")
     return dq, dk, dv
 
 
-def attn_bwd(q, k, v, dout, scale: float, causal: bool, window: int = -1
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, window: int = -1, block: int = 0
              ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Full dQ, dK, dV [B, H, n, d] in fp64."""
     B, H, n, d = q.shape
     rows = np.arange(B * H * n, dtype=np.int64)
-    dq, dk, dv = attn_bwd_rows(q, k, v, dout, scale, causal, window, rows, rows)
+    dq, dk, dv = attn_bwd_rows(q, k, v, dout, scale, causal, window, rows, rows, block)
     return dq.reshape(B, H, n, d), dk.reshape(B, H, n, d), dv.reshape(B, H, n, d)
 
 
@@ -263,10 +265,10 @@ def matmul(a: np.ndarray, b: np.ndarray, ta: bool = False, tb: bool = False) -> 
     return c
 
 
-def mask_row(n: int, i: int, causal: bool, window: int) -> np.ndarray:
+def mask_row(n: int, i: int, causal: bool, window: int, block: int = 0) -> np.ndarray:
     lib = _load()
     out = np.empty(n, dtype=np.uint8)
-    if lib.oracle_mask_row(n, i, int(bool(causal)), int(window), out.ctypes.data) != 0:
+    if lib.oracle_mask_row(n, i, int(bool(causal)), int(window), int(block), out.ctypes.data) != 0:
         raise ValueError("bad mask arguments")
     return out.astype(bool)
 

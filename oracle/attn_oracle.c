@@ -24,6 +24,10 @@
  *            max(0, i - w) <= j <= min(n - 1, i + w)  (the same page's local
  *            attention: each token attends to its w nearest neighbours on
  *            either side)
+ *   block-local (block b > 0, no window) : floor(j/b) is floor(i/b) or
+ *            floor(i/b) - 1, and j <= i as well when causal (the block-sparse
+ *            pattern of "Sparse & sub-quadratic attention", section "Escape 1":
+ *            attend within your block and the previous one)
  * Then, all in fp64 over the bf16-decoded inputs,
  *   s_ij  = scale * sum_c q_ic k_jc          for j in A(i)
  *   M_i   = max_{j in A(i)} s_ij
@@ -100,10 +104,14 @@ int oracle_matmul_f64(int64_t m, int64_t n, int64_t k, const double *A, int ta,
 }
 
 /* Is key j in A(i)? The one definition of the masks (see the top of the file). */
-static int allowed_pair(int64_t i, int64_t j, int causal, int64_t window)
+static int allowed_pair(int64_t i, int64_t j, int causal, int64_t window, int64_t block)
 {
     if (causal && j > i)
         return 0;
+    if (block > 0) {
+        const int64_t bi = i / block, bj = j / block;
+        return bj == bi || bj == bi - 1;
+    }
     if (window >= 0 && j < i - window)
         return 0;
     if (!causal && window >= 0 && j > i + window)
@@ -112,12 +120,12 @@ static int allowed_pair(int64_t i, int64_t j, int causal, int64_t window)
 }
 
 /* Explicit mask row: allowed[j] = 1 iff key j is in A(i). */
-int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned char *allowed)
+int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, int64_t block, unsigned char *allowed)
 {
-    if (n < 0 || i < 0 || i >= n || !allowed)
+    if (n < 0 || i < 0 || i >= n || !allowed || (block > 0 && window >= 0))
         return 1;
     for (int64_t j = 0; j < n; ++j)
-        allowed[j] = (unsigned char)allowed_pair(i, j, causal, window);
+        allowed[j] = (unsigned char)allowed_pair(i, j, causal, window, block);
     return 0;
 }
 
@@ -134,10 +142,12 @@ int oracle_mask_row(int64_t n, int64_t i, int causal, int64_t window, unsigned c
  */
 int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                              int64_t B, int64_t H, int64_t Hkv, int64_t n, int64_t d,
-                             double scale, int causal, int64_t window, int kernel,
+                             double scale, int causal, int64_t window, int64_t block, int kernel,
                              const int64_t *rows, int64_t nrows,
                              double *o, double *lse, double *weights)
 {
+    if (block > 0 && window >= 0)
+        return 1;
     if (!q || !k || !v || !o || (!rows && nrows) || B <= 0 || H <= 0 || n <= 0 || d <= 0)
         return 1;
     if (Hkv <= 0 || H % Hkv != 0)
@@ -175,7 +185,7 @@ int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_
                     for (int64_t j = 0; j < n; ++j)
                         allowed[j] = 1;
                 } else {
-                    oracle_mask_row(n, i, causal, window, allowed);
+                    oracle_mask_row(n, i, causal, window, block, allowed);
                 }
 
                 /* pass 1: scores of allowed keys and their maximum */
@@ -236,18 +246,18 @@ int oracle_attn_rows_gqa_f64(const uint16_t *q, const uint16_t *k, const uint16_
 /* Multi-head attention (Hkv = H) for a list of rows; arguments as above. */
 int oracle_attn_rows_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          int64_t B, int64_t H, int64_t n, int64_t d, double scale,
-                         int causal, int64_t window, int kernel,
+                         int causal, int64_t window, int64_t block, int kernel,
                          const int64_t *rows, int64_t nrows,
                          double *o, double *lse, double *weights)
 {
-    return oracle_attn_rows_gqa_f64(q, k, v, B, H, H, n, d, scale, causal, window, kernel,
+    return oracle_attn_rows_gqa_f64(q, k, v, B, H, H, n, d, scale, causal, window, block, kernel,
                                     rows, nrows, o, lse, weights);
 }
 
 /* Every row of every head: o is [B, H, n, d] fp64, lse is [B, H, n] fp64. */
 int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int64_t B, int64_t H, int64_t n, int64_t d, double scale,
-                        int causal, int64_t window, double *o, double *lse)
+                        int causal, int64_t window, int64_t block, double *o, double *lse)
 {
     if (B <= 0 || H <= 0 || n <= 0)
         return 1;
@@ -257,7 +267,7 @@ int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         return 2;
     for (int64_t r = 0; r < total; ++r)
         rows[r] = r;
-    int rc = oracle_attn_rows_f64(q, k, v, B, H, n, d, scale, causal, window,
+    int rc = oracle_attn_rows_f64(q, k, v, B, H, n, d, scale, causal, window, block,
                                   ORACLE_KERNEL_SOFTMAX, rows, total, o, lse, NULL);
     free(rows);
     return rc;
@@ -312,10 +322,10 @@ static double in_at(const void *p, int type, int64_t idx)
  * its key/value head (k, v); s and dp are n-long scratch. */
 static void bwd_row(const void *q, const void *k, const void *v, const void *dout, int type,
                     int64_t qbase, int64_t kbase, int64_t n, int64_t d, double scale, int causal,
-                    int64_t window, int64_t i, unsigned char *allowed, double *s, double *dp,
-                    double *lse_out, double *rowterm_out, double *dq)
+                    int64_t window, int64_t block, int64_t i, unsigned char *allowed, double *s,
+                    double *dp, double *lse_out, double *rowterm_out, double *dq)
 {
-    oracle_mask_row(n, i, causal, window, allowed);
+    oracle_mask_row(n, i, causal, window, block, allowed);
     double M = -INFINITY;
     for (int64_t j = 0; j < n; ++j) {
         if (!allowed[j])
@@ -375,9 +385,12 @@ static void bwd_row(const void *q, const void *k, const void *v, const void *dou
  */
 int oracle_attn_bwd_rows_gqa_f64(const void *q, const void *k, const void *v, const void *dout, int type,
                                  int64_t B, int64_t H, int64_t Hkv, int64_t n, int64_t d, double scale,
-                                 int causal, int64_t window, const int64_t *qrows, int64_t nq,
-                                 const int64_t *krows, int64_t nk, double *dq, double *dk, double *dv)
+                                 int causal, int64_t window, int64_t block, const int64_t *qrows,
+                                 int64_t nq, const int64_t *krows, int64_t nk, double *dq, double *dk,
+                                 double *dv)
 {
+    if (block > 0 && window >= 0)
+        return 1;
     if (!q || !k || !v || !dout || B <= 0 || H <= 0 || Hkv <= 0 || n <= 0 || d <= 0)
         return 1;
     if (H % Hkv != 0)
@@ -439,16 +452,16 @@ int oracle_attn_bwd_rows_gqa_f64(const void *q, const void *k, const void *v, co
             for (int64_t t = 0; t < nstat * n; ++t) {
                 const int64_t h = stat_head[t / n], i = t % n;
                 const int64_t kvh = (h / H) * Hkv + (h % H) / G;
-                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, i,
-                        allowed, s, dp, &lse[t], &rowterm[t], NULL);
+                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, block,
+                        i, allowed, s, dp, &lse[t], &rowterm[t], NULL);
             }
             /* 2. dQ of the requested query rows */
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < nq; ++r) {
                 const int64_t h = qrows[r] / n, i = qrows[r] % n;
                 const int64_t kvh = (h / H) * Hkv + (h % H) / G;
-                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, i,
-                        allowed, s, dp, NULL, NULL, dq + r * d);
+                bwd_row(q, k, v, dout, type, h * n * d, kvh * n * d, n, d, scale, causal, window, block,
+                        i, allowed, s, dp, NULL, NULL, dq + r * d);
             }
             /* 3. dK, dV of the requested key rows: sums over the query heads
              * of the group and the queries that attend to key j, with each
@@ -467,7 +480,7 @@ int oracle_attn_bwd_rows_gqa_f64(const void *q, const void *k, const void *v, co
                     const double *L = lse + slot[h] * n;
                     const double *R = rowterm + slot[h] * n;
                     for (int64_t i = 0; i < n; ++i) {
-                        if (!allowed_pair(i, j, causal, window))
+                        if (!allowed_pair(i, j, causal, window, block))
                             continue;
                         double sij = 0.0, dpij = 0.0;
                         for (int64_t c = 0; c < d; ++c) {
@@ -500,11 +513,11 @@ int oracle_attn_bwd_rows_gqa_f64(const void *q, const void *k, const void *v, co
 /* Multi-head form (Hkv = H); arguments as above. */
 int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const void *dout, int type,
                              int64_t B, int64_t H, int64_t n, int64_t d, double scale, int causal,
-                             int64_t window, const int64_t *qrows, int64_t nq, const int64_t *krows,
-                             int64_t nk, double *dq, double *dk, double *dv)
+                             int64_t window, int64_t block, const int64_t *qrows, int64_t nq,
+                             const int64_t *krows, int64_t nk, double *dq, double *dk, double *dv)
 {
-    return oracle_attn_bwd_rows_gqa_f64(q, k, v, dout, type, B, H, H, n, d, scale, causal, window, qrows,
-                                        nq, krows, nk, dq, dk, dv);
+    return oracle_attn_bwd_rows_gqa_f64(q, k, v, dout, type, B, H, H, n, d, scale, causal, window, block,
+                                        qrows, nq, krows, nk, dq, dk, dv);
 }
 
 /* ========================================================================

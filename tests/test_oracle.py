@@ -373,3 +373,48 @@ def test_symmetric_pair_count_closed_form():
         for w in (0, 1, 3, n - 1, n, 5 * n):
             direct = sum(min(n - 1, i + w) - max(0, i - w) + 1 for i in range(n))
             assert synth.attended_pairs_per_head(n, False, w) == direct
+
+
+# ---------------------------------------------------------------- block-local (block-sparse) mask
+
+def _block_keep(n, block, causal):
+    """The page's block-sparse pattern written with block indices: key j in
+    the query's block or the block before it (and j <= i if causal)."""
+    i = np.arange(n)[:, None] // block
+    j = np.arange(n)[None, :] // block
+    keep = (j == i) | (j == i - 1)
+    if causal:
+        keep &= np.arange(n)[None, :] <= np.arange(n)[:, None]
+    return keep
+
+
+@pytest.mark.parametrize("n,block", [(1, 4), (10, 1), (37, 4), (64, 16), (70, 128)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_matches_block_indices_and_brute_force(oracle_mod, n, block, causal):
+    keep = _block_keep(n, block, causal)
+    for i in range(n):
+        np.testing.assert_array_equal(oracle_mod.mask_row(n, i, causal, -1, block), keep[i])
+    q, k, v = synth.make_qkv(1, 2, n, 16, seed=n + block, q_std=2.0)
+    o, lse = oracle_mod.attn_fwd(q, k, v, 0.25, causal, -1, block)
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    S = np.where(keep, (Q @ np.swapaxes(K, -1, -2)) * 0.25, -np.inf)
+    M = S.max(axis=-1, keepdims=True)
+    E = np.exp(S - M)
+    np.testing.assert_allclose(o, (E / E.sum(-1, keepdims=True)) @ V, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, (M + np.log(E.sum(-1, keepdims=True)))[..., 0], rtol=0, atol=1e-12)
+    assert int(keep.sum()) == synth.attended_pairs_block(n, block, causal)
+
+
+def test_block_mask_special_cases(oracle_mod):
+    """b >= n: one block, so the mask is no mask (or causal); b = 1: keys i-1
+    and i, the causal window 1."""
+    q, k, v = synth.make_qkv(1, 2, 40, 16, seed=91, q_std=3.0)
+    for causal in (False, True):
+        a = oracle_mod.attn_fwd(q, k, v, 0.25, causal, -1, 64)
+        b = oracle_mod.attn_fwd(q, k, v, 0.25, causal, -1)
+        np.testing.assert_array_equal(a[0], b[0])
+        c = oracle_mod.attn_fwd(q, k, v, 0.25, causal, -1, 1)
+        d = oracle_mod.attn_fwd(q, k, v, 0.25, True, 1)
+        np.testing.assert_array_equal(c[0], d[0])
+    with pytest.raises(ValueError):
+        oracle_mod.attn_fwd(q, k, v, 0.25, True, 3, 8)  # a block mask takes no window

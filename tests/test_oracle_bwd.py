@@ -208,3 +208,22 @@ def test_gqa_bwd_equals_group_sum_of_multi_head_gradients(oracle_mod):
                                rtol=0, atol=1e-12)
     np.testing.assert_allclose(dv_g.reshape(B, Hkv, n, d), dv_m.reshape(B, Hkv, G, n, d).sum(axis=2),
                                rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("block", [1, 3, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_bwd_matches_autograd(oracle_mod, block, causal):
+    B, H, n, d = 1, 2, 21, 8
+    q, k, v, do = (_rand((B, H, n, d), s) for s in (71, 72, 73, 74))
+    i = torch.arange(n).view(n, 1)
+    j = torch.arange(n).view(1, n)
+    keep = ((j // block) == (i // block)) | ((j // block) == (i // block) - 1)
+    if causal:
+        keep &= j <= i
+    qa, ka, va = (x.clone().requires_grad_(True) for x in (q, k, v))
+    s = (qa @ ka.transpose(-1, -2)) * 0.5
+    o = s.masked_fill(~keep, float("-inf")).softmax(-1) @ va
+    (o * do).sum().backward()
+    dq, dk, dv = oracle_mod.attn_bwd(q, k, v, do, 0.5, causal, -1, block)
+    for got, ref in ((dq, qa.grad), (dk, ka.grad), (dv, va.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
