@@ -193,19 +193,19 @@ def cpu_baseline_leg(wl, o_gpu=None, lse_gpu=None, target_s: float = 15.0):
     from exact_softmax_attention_04_b200 import synth
     oracle.build()
     q, k, v = synth.make_inputs(wl)
-    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window)
+    pairs = synth.workload_pairs_per_head(wl)
     flops_per_row = 4.0 * wl.d * pairs / wl.n
     g = torch.Generator().manual_seed(2)
     total = wl.B * wl.H * wl.n
     # calibrate on a small sample, then size the sample to ~target_s seconds
     probe = torch.randint(0, total, (64,), generator=g).numpy()
     t0 = time.perf_counter()
-    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe, block=wl.block)
     dt = max(time.perf_counter() - t0, 1e-3)
     nrows = int(min(total, max(64, 64 * target_s / dt)))
     rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
     t0 = time.perf_counter()
-    o_ref, lse_ref = oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, rows)
+    o_ref, lse_ref = oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, rows, block=wl.block)
     dt = time.perf_counter() - t0
     out = {"value": nrows * flops_per_row / dt / 1e12, "unit": "TFLOP/s",
            "cores": oracle.num_threads(), "kind": "oracle",
@@ -234,24 +234,24 @@ def run_reference(args, wl, world, rank):
     from exact_softmax_attention_04_b200 import synth
     oracle.build()
     q, k, v = synth.make_inputs(wl)
-    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window)
+    pairs = synth.workload_pairs_per_head(wl)
     flops_per_row = 4.0 * wl.d * pairs / wl.n
     total = wl.B * wl.H * wl.n
     g = torch.Generator().manual_seed(3)
     # each step: a bounded sample sized so warmup + steps stay within ~2 minutes
     probe = torch.randint(0, total, (32,), generator=g).numpy()
     t0 = time.perf_counter()
-    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe)
+    oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, probe, block=wl.block)
     per_row = max((time.perf_counter() - t0) / 32, 1e-6)
     budget = args.reference_seconds / max(1, args.steps + args.warmup)
     nrows = int(max(8, min(total, budget / per_row)))
     samples = [np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
                for _ in range(args.steps + args.warmup)]
     for i in range(args.warmup):
-        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[i])
+        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[i], block=wl.block)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[args.warmup + i])
+        oracle.attn_rows_gqa(q, k, v, wl.scale, wl.causal, wl.window, samples[args.warmup + i], block=wl.block)
     dt = time.perf_counter() - t0
     value = args.steps * nrows * flops_per_row / dt / 1e12
     sample = f"{nrows} random query rows per step (seed 3) of {wl.name}, fp64 oracle"
@@ -313,7 +313,8 @@ def run_ours(args, wl, world, rank, local):
     flops = synth.unmasked_flops(wl)
 
     def step():
-        attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, stream=stream)
+        attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, stream=stream,
+                      block=wl.block)
 
     for _ in range(args.warmup):
         step()
@@ -359,8 +360,11 @@ def run_ours(args, wl, world, rank, local):
     # end to end through the host-buffer entry point: H2D of q,k,v, kernel,
     # D2H of o and lse, every step (that entry point takes equal head counts)
     e2e = None
-    if wl.kv_heads == wl.H:
+    if wl.kv_heads == wl.H and wl.block == 0:
         e2e = run_e2e(args, wl, q, k, v, o, lse, flops, dev, stream, world)
+    elif wl.block > 0:
+        e2e = {"value": None, "unit": "TFLOP/s",
+               "note": "block-local workload: the host-buffer entry point takes causal / window masks"}
     else:
         e2e = {"value": None, "unit": "TFLOP/s",
                "note": "grouped-query workload: the host-buffer entry point takes equal head counts"}
@@ -425,15 +429,15 @@ def run_bwd(args, wl, world, rank, local):
     do = synth.make_dout(wl.B, wl.H, wl.n, wl.d, seed=wl.seed)
     qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
     stream = torch.cuda.current_stream(dev)
-    o, lse = attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, stream=stream)
+    o, lse = attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, stream=stream, block=wl.block)
     ws = torch.empty(attn.bwd_workspace_bytes(wl.B, wl.H, wl.n, wl.d), dtype=torch.uint8, device=dev)
-    pairs = synth.attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H
+    pairs = synth.workload_pairs_per_head(wl) * wl.B * wl.H
     flops = 10 * wl.d * pairs
     grads = None
 
     def step():
         nonlocal grads
-        grads = attn.attn_bwd(qd, kd, vd, o, lse, dod, wl.scale, wl.causal, wl.window, workspace=ws,
+        grads = attn.attn_bwd(qd, kd, vd, o, lse, dod, wl.scale, wl.causal, wl.window, workspace=ws, block=wl.block,
                               stream=stream)
 
     for _ in range(args.warmup):
@@ -501,12 +505,12 @@ def run_bwd(args, wl, world, rank, local):
         flops_per_row = flops / total
         probe = torch.randint(0, total, (16,), generator=g).numpy()
         t0 = time.perf_counter()
-        oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, probe, [])
+        oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, probe, [], block=wl.block)
         dt = max(time.perf_counter() - t0, 1e-3)
         nrows = int(min(total, max(16, 16 * args.cpu_seconds / dt)))
         rows = np.sort(torch.randint(0, total, (nrows,), generator=g).numpy())
         t0 = time.perf_counter()
-        dq_ref, _, _ = oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, rows, [])
+        dq_ref, _, _ = oracle.attn_bwd_rows_gqa(q, k, v, do, wl.scale, wl.causal, wl.window, rows, [], block=wl.block)
         dt = time.perf_counter() - t0
         dq_gpu = grads[0].view(-1, wl.d)[torch.as_tensor(rows, device=dev)].float().cpu().numpy()
         diff = dq_gpu - dq_ref
@@ -628,7 +632,7 @@ def run_sweep(args):
     torch.cuda.set_device(0)
     bf16_peak, hbm_peak, peak_src = peaks()
     wls = [synth.SMALL_CAUSAL, synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072,
-           synth.GQA_N8192, synth.SYM_N16384] + synth.sweep()
+           synth.GQA_N8192, synth.SYM_N16384, synth.BLOCK_N16384] + synth.sweep()
     for wl in wls:
         q, k, v = synth.make_inputs(wl)
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -638,7 +642,7 @@ def run_sweep(args):
         min_bytes = 4 * q.numel() * 2 + lse.numel() * 4
         # L2 flush buffer (256 MB) between timed launches for small problems
         flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-        f = lambda: attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse)
+        f = lambda: attn.attn_fwd(qd, kd, vd, wl.scale, wl.causal, wl.window, out=o, lse=lse, block=wl.block)
         for _ in range(args.warmup):
             f()
         st = attn.sync_status()

@@ -30,7 +30,7 @@ ATTN_ERR_TOO_LARGE = 5
 EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_release",
            "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
            "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes", "attn_decode",
-           "attn_decode_workspace_bytes")
+           "attn_decode_workspace_bytes", "attn_fwd_blocklocal", "attn_bwd_blocklocal")
 
 
 class AttnError(RuntimeError):
@@ -56,6 +56,8 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_fwd.restype = i
     lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.attn_fwd_gqa.restype = i
+    lib.attn_fwd_blocklocal.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd_blocklocal.restype = i
     lib.attn_fwd_host.argtypes = fwd_args
     lib.attn_fwd_host.restype = i
     lib.attn_fwd_host_noalloc.argtypes = fwd_args
@@ -74,6 +76,9 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
                                  i, i, i, i, i, f, i, i, vp]
     lib.attn_bwd_gqa.restype = i
+    lib.attn_bwd_blocklocal.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                        i, i, i, i, i, f, i, i, vp]
+    lib.attn_bwd_blocklocal.restype = i
     lib.attn_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.attn_bwd_workspace_bytes.restype = i64
     lib.attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, f, vp]
@@ -135,15 +140,16 @@ def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, device: bool,
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
              causal: bool = False, window: int = -1, out: Optional[torch.Tensor] = None,
-             lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None
-             ) -> Tuple[torch.Tensor, torch.Tensor]:
+             lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+             block: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T) V and its per-row log-sum-exp, on the GPU.
 
     q: bf16 CUDA tensor [B, H, n, d]; k, v: [B, H, n, d], or [B, Hkv, n, d]
     with Hkv dividing H for grouped-query / multi-query attention (query
     head h reads key/value head h // (H // Hkv)). Contiguous, d in {64, 128}.
     causal / window: see include/attn.h (window >= 0 without causal is the
-    symmetric window i - window .. i + window).
+    symmetric window i - window .. i + window). block > 0 selects the
+    block-local mask instead of a window (own block and the previous one).
     Returns (o bf16 [B, H, n, d], lse fp32 [B, H, n]); enqueued on ``stream``
     (default: the current stream), asynchronous like any CUDA op.
     """
@@ -160,8 +166,14 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
         raise ValueError("out must be a contiguous bf16 tensor shaped like q")
     if lse.shape != (B, H, n) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 tensor [B, H, n]")
+    if block > 0 and window >= 0:
+        raise ValueError("a block-local mask takes no window")
     with torch.cuda.device(q.device):
-        if grouped:
+        if block > 0:
+            rc = lib().attn_fwd_blocklocal(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                           lse.data_ptr(), B, H, k.shape[1], n, d, float(scale),
+                                           int(bool(causal)), int(block), _stream_handle(stream))
+        elif grouped:
             rc = lib().attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     lse.data_ptr(), B, H, k.shape[1], n, d, float(scale),
                                     int(bool(causal)), int(window), _stream_handle(stream))
@@ -170,7 +182,7 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
                                 lse.data_ptr(), B, H, n, d, float(scale), int(bool(causal)),
                                 int(window), _stream_handle(stream))
     if rc != ATTN_OK:
-        raise AttnError(rc, "attn_fwd_gqa" if grouped else "attn_fwd")
+        raise AttnError(rc, "attn_fwd_blocklocal" if block > 0 else ("attn_fwd_gqa" if grouped else "attn_fwd"))
     return out, lse
 
 
@@ -184,7 +196,7 @@ def bwd_workspace_bytes(B: int, H: int, n: int, d: int) -> int:
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              lse: torch.Tensor, dout: torch.Tensor, scale: Optional[float] = None,
              causal: bool = False, window: int = -1, workspace: Optional[torch.Tensor] = None,
-             stream: Optional[torch.cuda.Stream] = None
+             stream: Optional[torch.cuda.Stream] = None, block: int = 0
              ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of the attention forward pass on the GPU.
 
@@ -213,15 +225,17 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace.device != q.device or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous tensor on q's device")
+    if block > 0 and window >= 0:
+        raise ValueError("a block-local mask takes no window")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), B, H, k.shape[1], n, d, float(scale),
+            int(bool(causal)), int(block if block > 0 else window), _stream_handle(stream))
     with torch.cuda.device(q.device):
-        rc = lib().attn_bwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                B, H, k.shape[1], n, d, float(scale), int(bool(causal)), int(window),
-                                _stream_handle(stream))
+        rc = (lib().attn_bwd_blocklocal if block > 0 else lib().attn_bwd_gqa)(*args)
     if rc != ATTN_OK:
-        raise AttnError(rc, "attn_bwd_gqa")
+        raise AttnError(rc, "attn_bwd_blocklocal" if block > 0 else "attn_bwd_gqa")
     return dq, dk, dv
 
 

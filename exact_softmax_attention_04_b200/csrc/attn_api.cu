@@ -73,6 +73,11 @@ int effective_window(int n, int window)
     return (window < 0 || window >= n - 1) ? -1 : window;
 }
 
+int effective_block(int n, int block)
+{
+    return (block <= 0 || block >= n) ? 0 : block;
+}
+
 int current_device(int *dev)
 {
     if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return ATTN_ERR_CUDA;
@@ -85,7 +90,7 @@ namespace {
 
 using namespace attn_host;
 
-bool g_smem_set[kMaxDevices][2] = {};
+bool g_smem_set[kMaxDevices][2][2] = {};  // [device][d==128][block mask]
 
 struct Staging {
     void *buf = nullptr;
@@ -115,10 +120,35 @@ int check_args(const void *q, const void *k, const void *v, const void *o, const
     return ATTN_OK;
 }
 
+// Sets the kernel's launch attributes once per device and checks its
+// register count against the split it was compiled for.
+template <int D, bool BLOCKMASK>
+int prepare_fwd(int dev)
+{
+    using Cfg = attn_sm100::FwdCfg<D>;
+    std::lock_guard<std::mutex> lk(g_mu);
+    bool &set = g_smem_set[dev][D == 128 ? 1 : 0][BLOCKMASK ? 1 : 0];
+    if (set) return ATTN_OK;
+    // The kernel moves registers between its warpgroups; that only works if it
+    // is launched with exactly the per-thread register count the split was
+    // computed for (else the raising warps wait forever). Refuse to launch a
+    // build that differs.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D, BLOCKMASK>) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D, BLOCKMASK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    set = true;
+    return ATTN_OK;
+}
+
 template <int D>
 int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int n,
                float scale, int causal, int window, cudaStream_t stream, int dev, int *status,
-               int Hkv = -1)
+               int Hkv = -1, int block = 0)
 {
     using Cfg = attn_sm100::FwdCfg<D>;
     auto enc = encoder();
@@ -130,25 +160,9 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     if (!encode_bhnd(enc, &mq, q, bh, n, D) || !encode_bhnd(enc, &mk, k, bhkv, n, D) ||
         !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mo, o, bh, n, D))
         return ATTN_ERR_CUDA;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = g_smem_set[dev][D == 128 ? 1 : 0];
-        if (!set) {
-            // The kernel moves registers between its warpgroups; that only
-            // works if it is launched with exactly the per-thread register
-            // count the split was computed for (else the raising warps wait
-            // forever). Refuse to launch a build that differs.
-            cudaFuncAttributes fa;
-            if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D>) != cudaSuccess)
-                return ATTN_ERR_CUDA;
-            if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
-            if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Cfg::SMEM_BYTES) != cudaSuccess)
-                return ATTN_ERR_CUDA;
-            set = true;
-        }
-    }
+    const bool blockmask = effective_block(n, block) > 0;
+    const int prc = blockmask ? prepare_fwd<D, true>(dev) : prepare_fwd<D, false>(dev);
+    if (prc != ATTN_OK) return prc;
     attn_sm100::FwdParams p;
     p.lse = lse;
     p.status = status;
@@ -160,8 +174,12 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
     p.window = effective_window(n, window);
+    p.block = effective_block(n, block);
     const unsigned grid = static_cast<unsigned>(bh * p.num_cta_tiles);
-    attn_sm100::attn_fwd_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    if (blockmask)
+        attn_sm100::attn_fwd_kernel<D, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else
+        attn_sm100::attn_fwd_kernel<D, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -195,6 +213,23 @@ extern "C" int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o
     if (d == 64)
         return launch_fwd<64>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status, Hkv);
     return launch_fwd<128>(q, k, v, o, lse, B, H, n, scale, causal, window, st, dev, status, Hkv);
+}
+
+extern "C" int attn_fwd_blocklocal(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   int B, int H, int Hkv, int n, int d, float scale, int causal, int block,
+                                   void *stream)
+{
+    if (block <= 0) return ATTN_ERR_INVALID;
+    const int rc = check_args(q, k, v, o, lse, B, H, n, d, scale, causal, -1, true, Hkv);
+    if (rc != ATTN_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    int *status = status_word(dev);
+    if (!status) return ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (d == 64)
+        return launch_fwd<64>(q, k, v, o, lse, B, H, n, scale, causal, -1, st, dev, status, Hkv, block);
+    return launch_fwd<128>(q, k, v, o, lse, B, H, n, scale, causal, -1, st, dev, status, Hkv, block);
 }
 
 extern "C" int attn_fwd_host(const void *q, const void *k, const void *v, void *o, float *lse, int B,

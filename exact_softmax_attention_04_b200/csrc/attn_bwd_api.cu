@@ -17,7 +17,7 @@ namespace {
 
 using namespace attn_host;
 
-bool g_bwd_set[kMaxDevices][2] = {};
+bool g_bwd_set[kMaxDevices][2][2] = {};  // [device][d==128][general]
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -92,7 +92,7 @@ int prepare_kernel(Kernel kernel, int smem_bytes, uint32_t regs_launch)
 template <int D>
 int launch_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int Hkv, int n,
-               float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+               float scale, int causal, int window, int block, cudaStream_t stream, int dev, int *status)
 {
     using KV = attn_sm100::BwdKVCfg<D>;
     using QC = attn_sm100::BwdQCfg<D>;
@@ -106,13 +106,18 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         !encode_bhnd(enc, &mdq, dq, bh, n, D) || !encode_bhnd(enc, &mdk, dk, bhkv, n, D) ||
         !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
+    const bool general = effective_block(n, block) > 0 || Hkv != H;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0];
+        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
         if (!set) {
-            int rc = prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
+            int rc = general
+                         ? prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, true>, KV::SMEM_BYTES, KV::REGS_LAUNCH)
+                         : prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, false>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
             if (rc == ATTN_OK)
-                rc = prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+                rc = general
+                         ? prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, true>, QC::SMEM_BYTES, QC::REGS_LAUNCH)
+                         : prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, false>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
             if (rc != ATTN_OK) return rc;
             set = true;
         }
@@ -145,15 +150,26 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
     p.window = effective_window(n, window);
+    p.block = effective_block(n, block);
 
     // 2. dK, dV: one CTA per key tile of each key/value head
-    attn_sm100::attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bhkv * p.num_k_tiles), KV::THREADS,
-                                          KV::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    const unsigned kv_grid = static_cast<unsigned>(bhkv * p.num_k_tiles);
+    if (general)
+        attn_sm100::attn_bwd_dkdv_kernel<D, true><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, p);
+    else
+        attn_sm100::attn_bwd_dkdv_kernel<D, false><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
     // 3. dQ: one CTA per query tile
-    attn_sm100::attn_bwd_dq_kernel<D><<<static_cast<unsigned>(bh * p.num_q_tiles), QC::THREADS,
-                                        QC::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+    const unsigned q_grid = static_cast<unsigned>(bh * p.num_q_tiles);
+    if (general)
+        attn_sm100::attn_bwd_dq_kernel<D, true><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdq, p);
+    else
+        attn_sm100::attn_bwd_dq_kernel<D, false><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -162,7 +178,8 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
 template <int D>
 int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o, const float *lse,
                      const void *dout, void *dq, void *dk, void *dv, char *ws, int B, int H, int Hkv,
-                     int n, float scale, int causal, int window, cudaStream_t stream, int dev, int *status)
+                     int n, float scale, int causal, int window, int block, cudaStream_t stream, int dev,
+                     int *status)
 {
     using Cfg = attn_sm100::FusedBwdCfg<D>;
     auto enc = encoder();
@@ -174,11 +191,15 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
         !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mdo, dout, bh, n, D) ||
         !encode_bhnd(enc, &mdk, dk, bhkv, n, D) || !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
+    const bool general = effective_block(n, block) > 0 || Hkv != H;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0];
+        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
         if (!set) {
-            const int rc = prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH);
+            const int rc =
+                general
+                    ? prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, true>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH)
+                    : prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, false>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH);
             if (rc != ATTN_OK) return rc;
             set = true;
         }
@@ -212,9 +233,14 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal;
     p.window = effective_window(n, window);
+    p.block = effective_block(n, block);
     const unsigned grid = static_cast<unsigned>(bhkv * p.num_k_tiles);
-    attn_sm100::attn_bwd_fused_kernel<D><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdk,
-                                                                                          mdv, macc, p);
+    if (general)
+        attn_sm100::attn_bwd_fused_kernel<D, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, macc, p);
+    else
+        attn_sm100::attn_bwd_fused_kernel<D, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, macc, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
     const int64_t count8 = bh * n * D / 8;
@@ -237,7 +263,7 @@ namespace {
 
 int bwd_entry(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
               void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int Hkv,
-              int n, int d, float scale, int causal, int window, void *stream)
+              int n, int d, float scale, int causal, int window, int block, void *stream)
 {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
     if (Hkv <= 0 || H <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
@@ -256,9 +282,9 @@ int bwd_entry(const void *q, const void *k, const void *v, const void *o, const 
     char *ws = static_cast<char *>(workspace);
     if (fused_for(d))
         return launch_bwd_fused<64>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, Hkv, n, scale, causal, window,
-                                    st, dev, status);
-    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, Hkv, n, scale, causal, window, st, dev,
-                           status);
+                                    block, st, dev, status);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, ws, B, H, Hkv, n, scale, causal, window, block,
+                           st, dev, status);
 }
 
 }  // namespace
@@ -269,7 +295,7 @@ extern "C" int attn_bwd(const void *q, const void *k, const void *v, const void 
                         int window, void *stream)
 {
     return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, H, n, d, scale, causal,
-                     window, stream);
+                     window, 0, stream);
 }
 
 extern "C" int attn_bwd_gqa(const void *q, const void *k, const void *v, const void *o, const float *lse,
@@ -278,5 +304,15 @@ extern "C" int attn_bwd_gqa(const void *q, const void *k, const void *v, const v
                             int window, void *stream)
 {
     return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, n, d, scale,
-                     causal, window, stream);
+                     causal, window, 0, stream);
+}
+
+extern "C" int attn_bwd_blocklocal(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                                   const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                                   size_t workspace_bytes, int B, int H, int Hkv, int n, int d, float scale,
+                                   int causal, int block, void *stream)
+{
+    if (block <= 0) return ATTN_ERR_INVALID;
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, n, d, scale,
+                     causal, -1, block, stream);
 }

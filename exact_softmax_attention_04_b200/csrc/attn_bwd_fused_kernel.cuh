@@ -56,6 +56,7 @@ struct FusedBwdParams {
     float scale_log2;    // scale * log2(e)
     int causal;
     int window;          // < 0: none
+    int block;           // > 0: block-local mask (see Mask)
 };
 
 template <int D>
@@ -187,7 +188,10 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------------------
 // 2. The main backward kernel.
-template <int D>
+// GENERAL: compiled for grouped-query heads (kv_heads < heads) or the
+// block-local mask (block > 0); the other instantiation handles multi-head
+// attention under the causal and window masks.
+template <int D, bool GENERAL>
 __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
     attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -237,11 +241,12 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
     const int k0 = kt * BN;
     const int n = p.n;
     int qlo, qhi;
-    query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
+    if constexpr (GENERAL)
+        query_tile_range(k0, Mask{n, p.causal, p.window, p.block}, qlo, qhi);
+    else
+        query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
     const int nq = qhi - qlo;  // >= 1: query k0 attends to key k0
-    const int nitems = G * nq;
-    auto item_q0 = [&](int it) { return (qlo + it % nq) * BM; };
-    auto item_bh = [&](int it) { return bh0 + it / nq; };
+    const int nitems = GENERAL ? G * nq : nq;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -290,12 +295,13 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
             tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bkv);
         }
         int issued = 0;
-        for (int it = 0; it < nitems; ++it) {
+        // (qi, g) = (it % nq, it / nq), kept by increment
+        for (int it = 0, qi = 0, g = 0; it < nitems; ++it, next_item<GENERAL>(qi, g, nq)) {
             const int s = it % NST;
             if (it >= NST && !__all_sync(0xffffffffu, wt.wait(q_empty(s), ((it / NST) & 1u) ^ 1u)))
                 break;
-            const int q0 = item_q0(it);
-            const int bh = item_bh(it);
+            const int q0 = (qlo + qi) * BM;
+            const int bh = bh0 + g;
 #ifdef ATTN_FAULT_BWD_DROP_FIRST_Q
             // Test hook (never defined in the library build): the first Q/dO
             // stage is never loaded, so the MMA warp's wait on it must expire
@@ -435,12 +441,13 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
                              f2u(u2f(v[4 * j + 2]) * sc), f2u(u2f(v[4 * j + 3]) * sc));
             }
         };
-        for (int it = 0; it < nitems; ++it) {
+        for (int it = 0, qi = 0, g = 0; it < nitems; ++it, next_item<GENERAL>(qi, g, nq)) {
             // all four warps take the same decision (they meet at named
             // barriers below)
             if (!named_bar_and(3, BM, wt.wait(dq_full, it & 1u))) break;
             tc_fence_after();
-            const int q0 = item_q0(it);
+            const int q0 = (qlo + qi) * BM;
+            const int bh = bh0 + g;
 #pragma unroll 1
             for (int hf = 0; hf < D / 64; ++hf) {
                 uint32_t va[32], vb[32];
@@ -459,8 +466,8 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
                 fence_proxy_async_smem();
                 named_bar_sync(3, BM);
                 if (issuer) {
-                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, item_bh(it));
-                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, item_bh(it));
+                    tma_reduce_add_3d(&tmdQacc, stage, 64 * hf, q0, bh);
+                    tma_reduce_add_3d(&tmdQacc, stage + BM * 128, 64 * hf + 32, q0, bh);
                     tma_store_commit();
                 }
             }
@@ -481,21 +488,34 @@ __global__ void __launch_bounds__(FusedBwdCfg<D>::THREADS, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
+        // Block mask: bounds that do not change along the query walk.
+        const Mask mk{n, p.causal, p.window, p.block};
+        const int key_first = mk.first_query(key), key_last = (key < n) ? mk.last_query(key) : -1;
+        const int tile_first = mk.first_query(min(k0 + BN - 1, n - 1)), tile_last = mk.last_query(k0);
+        const bool tile_ragged = k0 + BN > n;
         bool ok = true;
-        for (int it = 0; it < nitems; ++it) {
+        for (int it = 0, qi = 0, g = 0; it < nitems; ++it, next_item<GENERAL>(qi, g, nq)) {
             const int s = it % NST;
-            const int q0 = item_q0(it);
+            const int q0 = (qlo + qi) * BM;
             ok = __all_sync(0xffffffffu, wt.wait(s_full, it & 1u));
             if (!ok) break;
             tc_fence_after();
             // Allowed query columns of this key row: one interval [lo, hi].
-            const bool need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
-                                   (window >= 0 && q0 + BM - 1 > k0 + window) ||
-                                   (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
-            int lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
-            int hi = min(BM - 1, n - 1 - q0);
-            if (window >= 0) hi = min(hi, key + window - q0);
-            if (key >= n) hi = -1;
+            bool need_mask;
+            int lo, hi;
+            if constexpr (GENERAL) {
+                need_mask = tile_ragged || (q0 + BM > n) || tile_first > q0 || tile_last < q0 + BM - 1;
+                lo = key_first - q0;
+                hi = (key < n) ? key_last - q0 : -1;
+            } else {
+                need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
+                            (window >= 0 && q0 + BM - 1 > k0 + window) ||
+                            (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
+                lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
+                hi = min(BM - 1, n - 1 - q0);
+                if (window >= 0) hi = min(hi, key + window - q0);
+                if (key >= n) hi = -1;
+            }
             const uint32_t stat = sStat(s);
             float pf[64];
 #pragma unroll

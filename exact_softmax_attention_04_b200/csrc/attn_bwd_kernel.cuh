@@ -78,6 +78,7 @@ struct BwdParams {
     float scale_log2;    // scale * log2(e)
     int causal;
     int window;          // < 0: none
+    int block;           // > 0: block-local mask (see Mask)
 };
 
 // Launch shape shared by both main kernels.
@@ -227,9 +228,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // Query tiles [qlo, qhi) holding a query that attends to some key of the key
-// tile starting at k0 (k0 < n): causal queries start at the key tile's own
-// tile, a symmetric window starts them at k0 - window; any window ends them
-// at k0 + 127 + window.
+// tile starting at k0 (k0 < n). Causal and window masks only (the kernels'
+// specialisation without a block mask keeps this arithmetic).
 __device__ __forceinline__ void query_tile_range(int k0, int n, int causal, int window, int &qlo,
                                                  int &qhi)
 {
@@ -241,6 +241,31 @@ __device__ __forceinline__ void query_tile_range(int k0, int n, int causal, int 
         qhi = static_cast<int>(last / BM) + 1;
     }
 }
+
+// The same for any Mask (used with a block mask).
+__device__ __forceinline__ void query_tile_range(int k0, const Mask &mk, int &qlo, int &qhi)
+{
+    qlo = mk.first_query(k0) / BM;
+    qhi = mk.last_query(min(k0 + BN - 1, mk.n - 1)) / BM + 1;
+}
+
+// The key-tile kernels walk items it = 0, 1, ...: query tile qi = it % nq of
+// the group's head g = it / nq. WALK_GROUPS false: one head, qi = it (the
+// counters stay out of the instantiation for multi-head attention).
+template <bool WALK_GROUPS>
+__device__ __forceinline__ void next_item(int &qi, int &g, int nq)
+{
+    if constexpr (WALK_GROUPS) {
+        if (++qi == nq) {
+            qi = 0;
+            ++g;
+        }
+    } else {
+        ++qi;
+    }
+}
+
+
 
 // Dynamic shared memory base rounded up to 1 KB (the 128-byte swizzle atoms
 // need it); false if the slack does not allow it (never with the 1 KB of
@@ -255,8 +280,10 @@ __device__ __forceinline__ bool smem_base_1k(uint8_t *raw_ptr, uint32_t &base, u
 }
 
 // ---------------------------------------------------------------------------
-// 2. dK and dV.
-template <int D>
+// 2. dK and dV. GENERAL: compiled for grouped-query heads (kv_heads <
+// heads) or the block-local mask (block > 0); the other instantiation handles
+// multi-head attention under the causal and window masks.
+template <int D, bool GENERAL>
 __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -301,11 +328,12 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     const int G = p.heads / p.kv_heads;
     const int bh0 = (bkv / p.kv_heads) * p.heads + (bkv % p.kv_heads) * G;  // first query head
     int qlo, qhi;
-    query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
+    if constexpr (GENERAL)
+        query_tile_range(k0, Mask{n, p.causal, p.window, p.block}, qlo, qhi);
+    else
+        query_tile_range(k0, n, p.causal, p.window, qlo, qhi);
     const int nq = qhi - qlo;  // >= 1: query k0 attends to key k0
-    const int nitems = G * nq;
-    auto item_q0 = [&](int it) { return (qlo + it % nq) * BM; };
-    auto item_bh = [&](int it) { return bh0 + it / nq; };
+    const int nitems = GENERAL ? G * nq : nq;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -350,12 +378,13 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             tma_load_3d_if(leader, sV + b * BOX_BYTES, &tmV, kv_full, b * BOX_COLS, k0, bkv);
         }
         int issued = 0;
-        for (int it = 0; it < nitems; ++it) {
+        // (qi, g) = (it % nq, it / nq), kept by increment
+        for (int it = 0, qi = 0, g = 0; it < nitems; ++it, next_item<GENERAL>(qi, g, nq)) {
             const int s = it % NST;
             if (it >= NST && !__all_sync(0xffffffffu, wt.wait(q_empty(s), ((it / NST) & 1u) ^ 1u)))
                 break;
-            const int q0 = item_q0(it);
-            const int bh = item_bh(it);
+            const int q0 = (qlo + qi) * BM;
+            const int bh = bh0 + g;
 #ifdef ATTN_FAULT_BWD_DROP_FIRST_Q
             // Test hook (never defined in the library build): the first Q/dO
             // stage is never loaded, so the MMA warp's wait on it must expire
@@ -469,21 +498,36 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
+        // Block mask: bounds that do not change along the query walk (this
+        // key's attending queries, and the bounds every key of the tile
+        // shares).
+        const Mask mk{n, p.causal, p.window, p.block};
+        const int key_first = mk.first_query(key), key_last = (key < n) ? mk.last_query(key) : -1;
+        const int tile_first = mk.first_query(min(k0 + BN - 1, n - 1)), tile_last = mk.last_query(k0);
+        const bool tile_ragged = k0 + BN > n;
         bool ok = true;
-        for (int it = 0; it < nitems; ++it) {
+        for (int it = 0, qi = 0, g = 0; it < nitems; ++it, next_item<GENERAL>(qi, g, nq)) {
             const int s = it % NST;
-            const int q0 = item_q0(it);
+            const int q0 = (qlo + qi) * BM;
             ok = __all_sync(0xffffffffu, wt.wait(s_full, it & 1u));
             if (!ok) break;
             tc_fence_after();
             // Allowed query columns of this key row: one interval [lo, hi].
-            const bool need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
-                                   (window >= 0 && q0 + BM - 1 > k0 + window) ||
-                                   (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
-            const int lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
-            int hi = min(BM - 1, n - 1 - q0);
-            if (window >= 0) hi = min(hi, key + window - q0);
-            if (key >= n) hi = -1;
+            bool need_mask;
+            int lo, hi;
+            if constexpr (GENERAL) {
+                need_mask = tile_ragged || (q0 + BM > n) || tile_first > q0 || tile_last < q0 + BM - 1;
+                lo = key_first - q0;
+                hi = (key < n) ? key_last - q0 : -1;
+            } else {
+                need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
+                            (window >= 0 && q0 + BM - 1 > k0 + window) ||
+                            (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
+                lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
+                hi = min(BM - 1, n - 1 - q0);
+                if (window >= 0) hi = min(hi, key + window - q0);
+                if (key >= n) hi = -1;
+            }
             const uint32_t stat = sStat(s);
             float pf[64];
 #pragma unroll
@@ -593,7 +637,9 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
 
 // ---------------------------------------------------------------------------
 // 3. dQ.
-template <int D>
+// GENERAL as for attn_bwd_dkdv_kernel (here only the mask arithmetic
+// differs: the head mapping is the same for both).
+template <int D, bool GENERAL>
 __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -632,7 +678,10 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     const int q0 = qt * BM;
     const int n = p.n;
     int jlo, jhi;
-    key_tile_range(q0, n, p.causal, p.window, jlo, jhi);
+    if constexpr (GENERAL)
+        key_tile_range(q0, Mask{n, p.causal, p.window, p.block}, jlo, jhi);
+    else
+        key_tile_range(q0, n, p.causal, p.window, jlo, jhi);
     const int nkv = jhi - jlo;  // >= 1: key q0 is allowed for query q0
 
     if (threadIdx.x == 0) {
@@ -777,6 +826,10 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
+        // Block mask: bounds that do not change along the key walk.
+        const Mask mk{n, p.causal, p.window, p.block};
+        const int row_first = mk.first_key(row), row_last = mk.last_key(row);
+        const int tile_first = mk.first_key(q0 + BM - 1), tile_last = mk.last_key(q0);
         // this row's log2-domain LSE and delta (0 in rows past n)
         const size_t srow = static_cast<size_t>(bh) * p.n_pad + row;
         const float nl2 = -p.lse2[srow];
@@ -816,12 +869,16 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             // S(t) is in registers: the MMA warp may compute S(t+1)
             tc_fence_before();
             mbar_arrive(s_read);
-            const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
-                                   (window >= 0 && k0 < q0 + BM - 1 - window) ||
-                                   (!causal && window >= 0 && k0 + BN - 1 > q0 + window);
+            const bool need_mask =
+                GENERAL ? ((k0 + BN > n) || tile_first > k0 || tile_last < k0 + BN - 1)
+                          : ((k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
+                             (window >= 0 && k0 < q0 + BM - 1 - window) ||
+                             (!causal && window >= 0 && k0 + BN - 1 > q0 + window));
             // allowed key columns of this row: [lo, hi], key = k0 + column
-            const int hi = min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1), n - 1 - k0);
-            const int lo = (window >= 0) ? row - window - k0 : 0;
+            const int hi = GENERAL ? row_last - k0
+                                     : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
+                                           n - 1 - k0);
+            const int lo = GENERAL ? row_first - k0 : ((window >= 0) ? row - window - k0 : 0);
             float pf[64];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

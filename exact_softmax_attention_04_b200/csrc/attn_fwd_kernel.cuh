@@ -82,6 +82,7 @@ struct FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal;
     int window;        // < 0: none
+    int block;         // > 0: block-local mask with blocks of this many tokens
 };
 
 template <int D>
@@ -155,11 +156,56 @@ struct Waiter {
     }
 };
 
+// Every mask as intervals: query i attends to the keys [first_key(i),
+// last_key(i)], key j is attended by the queries [first_query(j),
+// last_query(j)]. Masks: causal (j <= i); a window w >= 0 (keys from i - w,
+// and up to i + w when not causal); a block-local mask with blocks of b
+// tokens (keys of the query's block and of the previous one, and j <= i when
+// causal). The host passes w <= n - 2 and b < n (wider ones allow the same
+// keys as no such mask) and never a window and a block together. All four
+// bounds are non-decreasing in their argument.
+struct Mask {
+    int n, causal, window, block;
+
+    __device__ __forceinline__ int first_key(int i) const
+    {
+        if (window >= 0) return max(0, i - window);
+        if (block > 0) return max(0, (i / block - 1) * block);
+        return 0;
+    }
+    __device__ __forceinline__ int last_key(int i) const
+    {
+        int64_t hi = static_cast<int64_t>(n) - 1;
+        if (causal)
+            hi = i;
+        else if (window >= 0)
+            hi = static_cast<int64_t>(i) + window;
+        else if (block > 0)
+            hi = (static_cast<int64_t>(i / block) + 1) * block - 1;
+        return static_cast<int>(min(hi, static_cast<int64_t>(n) - 1));
+    }
+    __device__ __forceinline__ int first_query(int j) const
+    {
+        if (causal) return j;
+        if (window >= 0) return max(0, j - window);
+        if (block > 0) return (j / block) * block;
+        return 0;
+    }
+    __device__ __forceinline__ int last_query(int j) const
+    {
+        int64_t hi = static_cast<int64_t>(n) - 1;
+        if (window >= 0)
+            hi = static_cast<int64_t>(j) + window;
+        else if (block > 0)
+            hi = (static_cast<int64_t>(j / block) + 2) * block - 1;
+        return static_cast<int>(min(hi, static_cast<int64_t>(n) - 1));
+    }
+};
+
 // Key tiles [jlo, jhi) holding at least one key allowed for some row of the
 // query tile starting at m0 (fully masked tiles are never visited). Empty when
-// the query tile lies past n. A window (window >= 0, at most n - 2: the host
-// turns wider windows into no window) limits keys to i - window and, when
-// not causal, to i + window.
+// the query tile lies past n. Causal and window masks only (the kernels'
+// specialisation without a block mask keeps this arithmetic).
 __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int window, int &jlo,
                                                int &jhi)
 {
@@ -175,6 +221,17 @@ __device__ __forceinline__ void key_tile_range(int m0, int n, int causal, int wi
     const int kbeg = (window >= 0) ? max(0, m0 - window) : 0;
     jlo = kbeg / BN;
     jhi = (kend + BN - 1) / BN;
+}
+
+// The same for any Mask (used with a block mask).
+__device__ __forceinline__ void key_tile_range(int m0, const Mask &mk, int &jlo, int &jhi)
+{
+    if (m0 >= mk.n) {
+        jlo = jhi = 0;
+        return;
+    }
+    jlo = mk.first_key(m0) / BN;
+    jhi = (mk.last_key(min(m0 + BM - 1, mk.n - 1)) + 1 + BN - 1) / BN;
 }
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
@@ -201,7 +258,9 @@ __device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float &y0, float
     y1 = u2f(f2u(p.y) + (f2u(t.y) << 23));
 }
 
-template <int D>
+// BLOCKMASK: compiled for the block-local mask (p.block > 0); the other
+// instantiation handles the causal and window masks.
+template <int D, bool BLOCKMASK>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -247,7 +306,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int n = p.n;
     int jlo_s[QT], jhi_s[QT];
 #pragma unroll
-    for (int s = 0; s < QT; ++s) key_tile_range(m0 + s * BM, n, p.causal, p.window, jlo_s[s], jhi_s[s]);
+    for (int s = 0; s < QT; ++s) {
+        if constexpr (BLOCKMASK)
+            key_tile_range(m0 + s * BM, Mask{n, p.causal, p.window, p.block}, jlo_s[s], jhi_s[s]);
+        else
+            key_tile_range(m0 + s * BM, n, p.causal, p.window, jlo_s[s], jhi_s[s]);
+    }
     // Union of the ranges: contiguous, starts with tile 0's, ends with the last
     // non-empty tile's.
     const int jlo = jlo_s[0];
@@ -440,6 +504,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const uint32_t p_base = lane_base + C::P_COL + s * C::P_STRIDE;
         const float sc = p.scale_log2;
         const int causal = p.causal, window = p.window;
+        // Block mask: bounds that do not change along the key walk (this
+        // row's allowed keys, and the bounds every row of the tile shares).
+        const Mask mk{n, p.causal, p.window, p.block};
+        const int row_first = mk.first_key(row), row_last = mk.last_key(row);
+        const int tile_first = mk.first_key(q0 + BM - 1), tile_last = mk.last_key(q0);
         const int my_jlo = jlo_s[s], my_jhi = jhi_s[s];
         float mx = -CUDART_INF_F;  // running max, log2 units
         float l = 0.f;             // running normaliser relative to mx
@@ -459,15 +528,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             }
 
             const int k0 = j * BN;
-            const bool need_mask = (k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
-                                   (window >= 0 && k0 < q0 + BM - 1 - window) ||
-                                   (!causal && window >= 0 && k0 + BN - 1 > q0 + window);
+            const bool need_mask =
+                BLOCKMASK ? ((k0 + BN > n) || tile_first > k0 || tile_last < k0 + BN - 1)
+                          : ((k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
+                             (window >= 0 && k0 < q0 + BM - 1 - window) ||
+                             (!causal && window >= 0 && k0 + BN - 1 > q0 + window));
             if (need_mask) {
                 // Allowed keys of this row form one interval; in tile columns:
                 // [lo, hi] with key = k0 + column.
-                const int hi = min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
-                                   n - 1 - k0);
-                const int lo = (window >= 0) ? row - window - k0 : 0;
+                const int hi = BLOCKMASK ? row_last - k0
+                                         : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
+                                               n - 1 - k0);
+                const int lo = BLOCKMASK ? row_first - k0 : ((window >= 0) ? row - window - k0 : 0);
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
                     if (c > hi || c < lo) sv[c] = f2u(-CUDART_INF_F);

@@ -36,6 +36,10 @@ bool encode_bhnd(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const vo
 // so kernel index arithmetic never meets a window wider than n.
 int effective_window(int n, int window);
 
+// The block size the kernels see: 0 (none) for block <= 0 and for blocks of
+// n tokens or more (one block: the same keys as no block mask).
+int effective_block(int n, int block);
+
 // The calling thread's current device, checked against kMaxDevices.
 int current_device(int *dev);
 

@@ -36,6 +36,7 @@ class Workload:
     q_std: float = 1.0
     seed: int = 0
     Hkv: int = 0      # key/value heads (grouped-query attention); 0 means H
+    block: int = 0    # > 0: block-local mask (own block and the previous one)
 
     @property
     def scale(self) -> float:
@@ -47,6 +48,8 @@ class Workload:
 
     @property
     def mask(self) -> str:
+        if self.block > 0:
+            return f"block{self.block}" + ("-causal" if self.causal else "")
         if self.window >= 0:
             return f"window{self.window}" if self.causal else f"symwindow{self.window}"
         return "causal" if self.causal else "none"
@@ -103,9 +106,15 @@ def attended_pairs_block(n: int, block: int, causal: bool) -> int:
     return total
 
 
+def workload_pairs_per_head(wl: "Workload") -> int:
+    if wl.block > 0:
+        return attended_pairs_block(wl.n, wl.block, wl.causal)
+    return attended_pairs_per_head(wl.n, wl.causal, wl.window)
+
+
 def unmasked_flops(wl: "Workload") -> int:
     """4*d FLOPs per attended pair (2*d for QK^T, 2*d for PV), times B*H."""
-    return 4 * wl.d * attended_pairs_per_head(wl.n, wl.causal, wl.window) * wl.B * wl.H
+    return 4 * wl.d * workload_pairs_per_head(wl) * wl.B * wl.H
 
 
 def make_qkv(B: int, H: int, n: int, d: int, seed: int = 0, q_std: float = 1.0, Hkv: int = 0
@@ -169,6 +178,9 @@ GQA_N8192 = Workload("B1-H64-Hkv8-n8192-d128-causal", 1, 64, 8192, 128, True, Hk
 # Symmetric local window (each token sees 256 neighbours on either side, the
 # 512-token span of Longformer-style local attention), d = 64, 16k tokens.
 SYM_N16384 = Workload("B2-H16-n16384-d64-symwindow256", 2, 16, 16384, 64, False, 256)
+# Block-local mask (own block and the previous one) with 512-token blocks,
+# d = 128, 16k tokens: the block-sparse pattern of the sub-quadratic page.
+BLOCK_N16384 = Workload("B2-H16-n16384-d128-block512", 2, 16, 16384, 128, False, block=512)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -250,7 +262,8 @@ def sweep() -> List[Workload]:
 
 
 def by_name(name: str) -> Optional[Workload]:
-    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072, GQA_N8192, SYM_N16384] + sweep():
+    for wl in [SMALL_CAUSAL, FULL_N8192, WINDOW_N32768, CAUSAL_N131072, GQA_N8192, SYM_N16384,
+               BLOCK_N16384] + sweep():
         if wl.name == name:
             return wl
     return None

@@ -29,7 +29,9 @@
  *                              (symmetric local window: each token attends to
  *                              its window nearest neighbours on either side;
  *                              local attention section of the same page)
- * A window of n - 1 or more allows the same keys as no window.
+ * A window of n - 1 or more allows the same keys as no window. The
+ * block-local mask has entry points of its own (attn_fwd_blocklocal,
+ * attn_bwd_blocklocal).
  *
  * Layout: Q, K, V and O are bf16, contiguous [B, H, n, d] (token-major inside
  * each head, d fastest). LSE is fp32, contiguous [B, H, n], natural-log units.
@@ -112,6 +114,23 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
 ATTN_API int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, float *lse,
                           int B, int H, int Hkv, int n, int d, float scale, int causal,
                           int window, void *stream);
+
+/*
+ * attn_fwd_blocklocal - the forward pass with the block-local mask: with
+ * blocks of `block` consecutive tokens, query i attends to the keys of its
+ * own block and of the previous one, floor(j/block) in {floor(i/block) - 1,
+ * floor(i/block)}, and only to j <= i when causal = 1 (the block-sparse
+ * pattern of "Sparse & sub-quadratic attention", section "Escape 1":
+ * attend within your block and the previous one). A block of n tokens or
+ * more is one block: the same keys as attn_fwd without a window.
+ *
+ *   block  : >= 1 (else ATTN_ERR_INVALID)
+ *   Hkv    : key/value heads, as attn_fwd_gqa (Hkv = H for multi-head)
+ * Everything else as attn_fwd_gqa.
+ */
+ATTN_API int attn_fwd_blocklocal(const void *q, const void *k, const void *v, void *o,
+                                 float *lse, int B, int H, int Hkv, int n, int d, float scale,
+                                 int causal, int block, void *stream);
 
 /*
  * attn_fwd_host - the same operation on HOST buffers, copies included.
@@ -230,6 +249,17 @@ ATTN_API int attn_bwd_gqa(const void *q, const void *k, const void *v, const voi
                           const float *lse, const void *dout, void *dq, void *dk, void *dv,
                           void *workspace, size_t workspace_bytes, int B, int H, int Hkv, int n,
                           int d, float scale, int causal, int window, void *stream);
+
+/*
+ * attn_bwd_blocklocal - the backward pass of attn_fwd_blocklocal: arguments
+ * as attn_bwd_gqa with the block-local mask of attn_fwd_blocklocal in place
+ * of the window (block >= 1, else ATTN_ERR_INVALID).
+ */
+ATTN_API int attn_bwd_blocklocal(const void *q, const void *k, const void *v, const void *o,
+                                 const float *lse, const void *dout, void *dq, void *dk,
+                                 void *dv, void *workspace, size_t workspace_bytes, int B,
+                                 int H, int Hkv, int n, int d, float scale, int causal,
+                                 int block, void *stream);
 
 /* Device workspace bytes attn_bwd (and attn_bwd_gqa, with the query head
  * count H) needs for this shape, or -1 if the shape is invalid or

@@ -205,3 +205,23 @@ def test_bwd_gqa_entry_point_rejects_bad_head_counts(attn):
         rc = lib.attn_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40,
                               1, 8, Hkv, 128, 64, 0.125, 1, -1, None)
         assert rc == attn.ATTN_ERR_INVALID, Hkv
+
+
+def test_blocklocal_entry_points_reject_bad_blocks(attn):
+    lib = attn.lib()
+    for block in (0, -5):
+        assert lib.attn_fwd_blocklocal(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 8, 128, 64, 0.125, 1, block,
+                                       None) == attn.ATTN_ERR_INVALID
+        assert lib.attn_bwd_blocklocal(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40,
+                                       1, 8, 8, 128, 64, 0.125, 1, block, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_blocklocal(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 3, 128, 64, 0.125, 1, 64,
+                                   None) == attn.ATTN_ERR_INVALID   # 3 does not divide 8
+    assert lib.attn_fwd_blocklocal(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 8, 128, 96, 0.125, 1, 64,
+                                   None) == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_block_pair_count_workload(attn):
+    from exact_softmax_attention_04_b200 import synth
+    wl = synth.BLOCK_N16384
+    # 32 blocks of 512: block 0 sees itself (512 keys), later blocks 1024 keys
+    assert synth.workload_pairs_per_head(wl) == 512 * 512 + 31 * 512 * 1024

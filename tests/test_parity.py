@@ -205,3 +205,41 @@ def test_symmetric_window_closed_forms(attn, d):
         lo, hi = max(0, i - w), min(n - 1, i + w)
         assert (o[..., i, :] - vf[..., lo:hi + 1, :].mean(dim=-2)).abs().max() <= 2e-2
         assert (lse[..., i] - np.log(hi - lo + 1)).abs().max() <= 1e-3
+
+
+# ---------------------------------------------------------------- block-local mask
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [1, 64, 100, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_small_in_full(attn, oracle_mod, d, block, causal):
+    n = 600
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=block + d, q_std=4.0 if causal else 1.0)
+    sc = 1.0 / np.sqrt(d)
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), sc, causal, -1, block=block)
+    assert attn.sync_status() == attn.ATTN_OK
+    o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, sc, causal, -1, block)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"block{block} d{d} c{causal}")
+
+
+def test_block_mask_gqa(attn, oracle_mod):
+    B, H, Hkv, n, d = 2, 8, 2, 500, 128
+    q, k, v = synth.make_qkv(B, H, n, d, seed=95, Hkv=Hkv)
+    sc = 1.0 / np.sqrt(d)
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), sc, True, -1, block=160)
+    assert attn.sync_status() == attn.ATTN_OK
+    rows = np.arange(B * H * n)
+    o_ref, lse_ref = oracle_mod.attn_rows_gqa(q, k, v, sc, True, -1, rows, block=160)
+    assert_close(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1), o_ref, lse_ref, "gqa block")
+
+
+def test_block_workload_sampled(attn, oracle_mod):
+    wl = synth.BLOCK_N16384
+    q, k, v = synth.make_inputs(wl)
+    o, lse = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), wl.scale, wl.causal, wl.window, block=wl.block)
+    assert attn.sync_status() == attn.ATTN_OK
+    rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=16, bound_every=4, edge=16)
+    idx = torch.as_tensor(rows, device=o.device)
+    o_ref, lse_ref, _ = oracle_mod.attn_rows(q, k, v, wl.scale, wl.causal, wl.window, rows, block=wl.block)
+    assert_close(o.view(-1, wl.d)[idx].float().cpu().numpy(), lse.view(-1)[idx].cpu().numpy(), o_ref, lse_ref,
+                 wl.name)

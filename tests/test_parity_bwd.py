@@ -166,3 +166,23 @@ def test_gqa_bwd_equals_group_sums_of_multi_head(attn, d):
     for a, b in ((g[1], m[1]), (g[2], m[2])):
         ref = b.float().view(B, Hkv, G, n, d).sum(dim=2)
         assert (a.float() - ref).abs().max().item() <= 2e-2 * ref.abs().max().item()
+
+
+# ---------------------------------------------------------------- block-local mask
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block,causal", [(1, True), (64, False), (100, True), (256, False), (300, True)])
+@pytest.mark.parametrize("H,Hkv", [(2, 2), (4, 2)])
+def test_block_mask_bwd_small_in_full(attn, oracle_mod, d, block, causal, H, Hkv):
+    B, n = 1, 520
+    q, k, v = synth.make_qkv(B, H, n, d, seed=block + d + H, q_std=2.0, Hkv=Hkv)
+    do = synth.make_dout(B, H, n, d, seed=block + d + H)
+    sc = 1.0 / np.sqrt(d)
+    qc, kc, vc, doc = (x.cuda() for x in (q, k, v, do))
+    o, lse = attn.attn_fwd(qc, kc, vc, sc, causal, -1, block=block)
+    grads = attn.attn_bwd(qc, kc, vc, o, lse, doc, sc, causal, -1, block=block)
+    assert attn.sync_status() == attn.ATTN_OK
+    refs = oracle_mod.attn_bwd_rows_gqa(q, k, v, do, sc, causal, -1, np.arange(B * H * n),
+                                        np.arange(B * Hkv * n), block=block)
+    assert_grads_close([g.float().cpu().numpy().reshape(-1, d) for g in grads], refs,
+                       f"block{block} c{causal} H{H} Hkv{Hkv} d{d}")
