@@ -233,6 +233,9 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
             for (int kk = 0; kk < C::KPS; ++kk) {
                 const int k = psub * C::KPS + kk;
+                // slots past the cache: P is 0, but the slot may hold NaN
+                // (0 * NaN would reach O), so it is skipped
+                if (slot0 + k >= s1) continue;
                 const uint32_t addr = sV(s) + (pc / 8) * C::BOX_BYTES_T + k * 128 +
                                       ((static_cast<uint32_t>(pc % 8) ^ static_cast<uint32_t>(k & 7)) * 16);
                 uint4 vw;

@@ -1,9 +1,11 @@
 """Decode against rolling caches (through the C ABI) against the fp64 oracle.
 
 Small problems cover every grouped-query ratio, head size, partially filled
-and wrapped caches, cache sizes that are not a multiple of the 64-slot tile,
-and mixed positions within a batch; the full-size workload (64 sequences at
-position 32767 against 4096-slot caches) is compared on every row.
+and wrapped caches, cache sizes that are not a multiple of the 64- or
+128-slot tile (head size 64 and 128 run different kernels), mixed positions
+within a batch, and caches whose unused slots hold NaN; the full-size
+workload (64 sequences at position 32767 against 4096-slot caches) is
+compared on every row.
 """
 import numpy as np
 import pytest
@@ -34,7 +36,7 @@ def _gpu(attn, q, kc, vc, pos, scale=None):
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (8, 2), (8, 1)])
-@pytest.mark.parametrize("W", [1, 63, 64, 65, 200, 1024])
+@pytest.mark.parametrize("W", [1, 63, 64, 65, 127, 128, 129, 200, 1024])
 def test_decode_small_in_full(attn, oracle_mod, d, H, Hkv, W):
     B = 4
     q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=W * 3 + H + d, q_std=2.0)
@@ -68,3 +70,37 @@ def test_decode_full_size_workload_every_row(attn, oracle_mod):
                  o_ref.reshape(-1, wl.d), lse_ref.reshape(-1), wl.name)
     o2, l2 = _gpu(attn, q, kc, vc, [wl.pos] * wl.B, wl.scale)
     assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("W,pos", [(300, [0, 130, 255, 299]), (4096, [5, 1000, 2047, 2048]),
+                                   (2500, [1, 127, 128, 129])])
+def test_decode_unused_slots_hold_nan(attn, oracle_mod, d, W, pos):
+    """Slots no position has reached yet may hold anything, NaN included: the
+    result depends on the cached positions only (several splits of the slots
+    lie wholly or partly past them)."""
+    B, H, Hkv = len(pos), 8, 2
+    q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=W + d, q_std=2.0)
+    for b, t in enumerate(pos):
+        kc[b, :, t + 1:] = float("nan")
+        vc[b, :, t + 1:] = float("nan")
+    sc = 1.0 / np.sqrt(d)
+    o, lse = _gpu(attn, q, kc, vc, pos, sc)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    o_ref, lse_ref = oracle_mod.attn_decode(q, kc, vc, pos, sc)
+    assert_close(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1),
+                 o_ref.reshape(-1, d), lse_ref.reshape(-1), f"nan-slots W{W} d{d}")
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (8, 1), (16, 2)])
+def test_decode_d128_many_splits_mixed_positions(attn, oracle_mod, H, Hkv):
+    """Few (sequence, kv head) pairs, so the 4096 slots are cut into many
+    splits; positions from one slot to a wrapped cache."""
+    B, W, d = 3, 4096, 128
+    q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=H * 7 + Hkv, q_std=3.0)
+    pos = [0, 2049, 40000]
+    sc = 1.0 / np.sqrt(d)
+    o, lse = _gpu(attn, q, kc, vc, pos, sc)
+    o_ref, lse_ref = oracle_mod.attn_decode(q, kc, vc, pos, sc)
+    assert_close(o.float().cpu().numpy().reshape(-1, d), lse.cpu().numpy().reshape(-1),
+                 o_ref.reshape(-1, d), lse_ref.reshape(-1), f"splits H{H} Hkv{Hkv}")
