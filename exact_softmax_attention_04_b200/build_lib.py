@@ -15,8 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn_b200.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("attn_api.cu", "attn_bwd_api.cu", "attn_decode_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "attn_bwd_kernel.cuh",
-                                            "attn_bwd_fused_kernel.cuh", "attn_decode_kernel.cuh",
-                                            "attn_decode_tc_kernel.cuh", "sm100.cuh",
+                                            "attn_bwd_fused_kernel.cuh", "attn_decode_kernel.cuh", "sm100.cuh",
                                             "attn_host.h")] + [
     os.path.join(ROOT, "include", "attn.h")]
 

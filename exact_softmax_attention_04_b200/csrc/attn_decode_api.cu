@@ -10,7 +10,6 @@
 
 #include "attn.h"
 #include "attn_decode_kernel.cuh"
-#include "attn_decode_tc_kernel.cuh"
 #include "attn_host.h"
 
 namespace {
@@ -19,30 +18,12 @@ using namespace attn_host;
 
 bool g_dec_set[kMaxDevices][2][4] = {};  // [device][d==128][log2 G]
 
-// Splits of the W slots per (batch, kv head): about ATTN_DECODE_CTAS_PER_SM
-// CTAs per SM of a 148-SM B200 in total, each split a whole number of
-// 64-slot tiles.
-#ifndef ATTN_DECODE_CTAS_PER_SM
-#define ATTN_DECODE_CTAS_PER_SM 4
-#endif
+// Splits of the W slots per (batch, kv head): whole 128-slot tiles, two
+// resident CTAs per SM of a 148-SM B200. Minimises waves x (tiles per split
+// + 1), the +1 standing for a CTA's pipeline fill and drain.
 void choose_splits(int64_t bkv, int W, int *nsplit, int *chunk)
 {
     const int tiles = (W + attn_sm100::DEC_TK - 1) / attn_sm100::DEC_TK;
-    const int64_t target = ATTN_DECODE_CTAS_PER_SM * 148;
-    int64_t ns = (target + bkv - 1) / bkv;
-    if (ns < 1) ns = 1;
-    if (ns > tiles) ns = tiles;
-    const int tiles_per = static_cast<int>((tiles + ns - 1) / ns);
-    *chunk = tiles_per * attn_sm100::DEC_TK;
-    *nsplit = (W + *chunk - 1) / *chunk;
-}
-
-// Splits for the tensor-core kernel (head size 128): whole 128-slot tiles,
-// two resident CTAs per SM of a 148-SM B200. Minimises waves x (tiles per
-// split + 1), the +1 standing for a CTA's pipeline fill and drain.
-void choose_splits_tc(int64_t bkv, int W, int *nsplit, int *chunk)
-{
-    const int tiles = (W + attn_sm100::DTC_TK - 1) / attn_sm100::DTC_TK;
     const int64_t resident = 2 * 148;
     int best_per = tiles;
     double best_cost = -1.0;
@@ -55,16 +36,8 @@ void choose_splits_tc(int64_t bkv, int W, int *nsplit, int *chunk)
             best_per = per;
         }
     }
-    *chunk = best_per * attn_sm100::DTC_TK;
+    *chunk = best_per * attn_sm100::DEC_TK;
     *nsplit = (W + *chunk - 1) / *chunk;
-}
-
-void splits_for(int d, int64_t bkv, int W, int *nsplit, int *chunk)
-{
-    if (d == 128)
-        choose_splits_tc(bkv, W, nsplit, chunk);
-    else
-        choose_splits(bkv, W, nsplit, chunk);
 }
 
 int check_decode_args(int B, int H, int Hkv, int W, int d, float scale)
@@ -84,20 +57,21 @@ int check_decode_args(int B, int H, int Hkv, int W, int d, float scale)
 size_t decode_workspace(int B, int H, int Hkv, int W, int d)
 {
     int nsplit = 0, chunk = 0;
-    splits_for(d, static_cast<int64_t>(B) * Hkv, W, &nsplit, &chunk);
+    (void)d;
+    choose_splits(static_cast<int64_t>(B) * Hkv, W, &nsplit, &chunk);
     return static_cast<size_t>(nsplit) * B * H * (d + 2) * 4;
 }
 
 // Cache [bkv, W, d] bf16 as a 3-D tensor (d fastest), boxes of 64 columns x
-// box_rows slots x 1, 128-byte swizzle; slots past W read as zero.
+// 128 slots x 1, 128-byte swizzle; slots past W read as zero.
 bool encode_cache(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap *m, const void *ptr, int64_t bkv,
-                  int64_t W, int64_t d, int box_rows)
+                  int64_t W, int64_t d)
 {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(W),
                           static_cast<cuuint64_t>(bkv)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(W * d * 2)};
     cuuint32_t box[3] = {static_cast<cuuint32_t>(attn_sm100::BOX_COLS),
-                         static_cast<cuuint32_t>(box_rows), 1};
+                         static_cast<cuuint32_t>(attn_sm100::DEC_TK), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -114,24 +88,14 @@ int launch_decode(const void *q, const void *kc, const void *vc, const int *pos,
     if (!enc) return ATTN_ERR_CUDA;
     const int64_t bkv = static_cast<int64_t>(B) * Hkv;
     CUtensorMap mk, mv;
-    // head size 128: the tensor-core kernel with 128-slot tiles
-    constexpr bool TC = (D == 128);
-    using TcCfg = attn_sm100::DecTcCfg<G>;
-    const int box_rows = TC ? attn_sm100::DTC_TK : attn_sm100::DEC_TK;
-    if (!encode_cache(enc, &mk, kc, bkv, W, D, box_rows) || !encode_cache(enc, &mv, vc, bkv, W, D, box_rows))
-        return ATTN_ERR_CUDA;
+    if (!encode_cache(enc, &mk, kc, bkv, W, D) || !encode_cache(enc, &mv, vc, bkv, W, D)) return ATTN_ERR_CUDA;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         bool &set = g_dec_set[dev][D == 128 ? 1 : 0][G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3];
         if (!set) {
-            cudaError_t e;
-            if constexpr (TC)
-                e = cudaFuncSetAttribute(attn_sm100::attn_decode_tc_kernel<G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg::SMEM_BYTES);
-            else
-                e = cudaFuncSetAttribute(attn_sm100::attn_decode_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-            if (e != cudaSuccess) return ATTN_ERR_CUDA;
+            if (cudaFuncSetAttribute(attn_sm100::attn_decode_kernel<D, G>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+                return ATTN_ERR_CUDA;
             set = true;
         }
     }
@@ -143,13 +107,10 @@ int launch_decode(const void *q, const void *kc, const void *vc, const int *pos,
     p.H = H;
     p.Hkv = Hkv;
     p.W = W;
-    splits_for(D, bkv, W, &p.nsplit, &p.chunk);
+    choose_splits(bkv, W, &p.nsplit, &p.chunk);
     p.scale_log2 = scale * 1.4426950408889634f;
     const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(bkv));
-    if constexpr (TC)
-        attn_sm100::attn_decode_tc_kernel<G><<<grid, attn_sm100::DTC_THREADS, TcCfg::SMEM_BYTES, stream>>>(mk, mv, p);
-    else
-        attn_sm100::attn_decode_kernel<D, G><<<grid, attn_sm100::DEC_THREADS, Cfg::SMEM_BYTES, stream>>>(mk, mv, p);
+    attn_sm100::attn_decode_kernel<D, G><<<grid, attn_sm100::DEC_THREADS, Cfg::SMEM_BYTES, stream>>>(mk, mv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     const int rows = B * H;
     attn_sm100::attn_decode_combine_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(

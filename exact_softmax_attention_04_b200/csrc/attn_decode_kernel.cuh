@@ -9,26 +9,41 @@
 // Query head h reads key/value head h / G, G = H / Hkv (grouped-query
 // attention, "week17 efficiency attention", MQA / GQA section).
 //
-// The step reads every cached key and value once and does 4*d FLOPs per
-// (query head, key): it is bound by HBM bandwidth, so it runs on the CUDA
-// cores and is organised around streaming the caches:
-//   attn_decode_kernel: one CTA per (split of the slots, batch * kv head).
-//     The CTA's G query rows sit in shared memory (fp32); K and V tiles of 64
-//     slots stream in by TMA (128-byte swizzle) through a two-stage ring.
-//     Per tile: scores (thread = key; its q rows come as broadcasts), an
-//     online softmax per query head (running max and sum), and O += P V
-//     (thread = 8 columns of d x a subset of the tile's keys, all G heads).
-//     The CTA writes its unnormalised partial O, running max and sum.
+// The step reads every cached key and value once for 4*d FLOPs per (query
+// head, key): it is bound by HBM bandwidth, and what decides how close it
+// gets is the instruction count per cached byte. Both contractions of a
+// 128-slot tile are therefore tcgen05 MMAs (a tile costs a few hundred
+// instructions; on the CUDA cores every key is converted and multiplied once
+// per query head):
+//   S^T  = K_tile q^T     M = 128 slots, N = 16 (the G query heads of the
+//                         group, zero rows up to 16), K = d; fp32 in TMEM
+//                         with lane = slot;
+//   O^T += V_tile^T P^T   M = d, N = 16, K = 128 slots: the V tile as it
+//                         lands from TMA is the MN-major A operand, P^T a
+//                         16-row K-major operand written by the softmax. At
+//                         d = 64 the accumulator has M = 64 rows, which TMEM
+//                         holds as 16 lanes of each 32-lane quarter (row
+//                         16 q + i in lane 32 q + i).
+//   attn_decode_kernel: one CTA per (split of the slots, batch * kv head),
+//     192 threads:
+//     warp 0     TMA producer: K_0, V_0, K_1, V_1, ... through one ring of
+//                96 KB (3 stages of 32 KB tiles at d = 128, 6 of 16 KB at 64);
+//     warp 1     TMEM owner and MMA issuer, order S(0), S(1), PV(0), S(2),
+//                PV(1), ... so the next scores are ready when the softmax
+//                ends a tile;
+//     warps 2-5  softmax, one thread per slot (= TMEM lane): per query head
+//                the tile max over 128 slots (shuffles, then the four warps
+//                through shared memory), running max, per-thread partial
+//                sums, P^T into shared memory (bf16), and the rescale of O^T
+//                in TMEM when a head's max grows. They finish with O^T.
+//     The CTA writes its unnormalised partial O, running max and sum. About
+//     110 KB of shared memory and 64 TMEM columns: two CTAs per SM.
 //   attn_decode_combine_kernel: merges the splits of every (b, h) with the
 //     log-sum-exp rule and writes O (bf16) and LSE.
 #pragma once
 #include "attn_fwd_kernel.cuh"
 
 namespace attn_sm100 {
-
-constexpr int DEC_TK = 64;         // slots per tile (TMA box rows)
-constexpr int DEC_THREADS = 256;
-constexpr int DEC_NST = 2;         // K/V ring stages
 
 struct DecodeParams {
     const __nv_bfloat16 *q;  // [B, H, D]
@@ -41,54 +56,66 @@ struct DecodeParams {
     float scale_log2;        // scale * log2(e)
 };
 
+constexpr int DEC_TK = 128;       // slots per tile
+constexpr int DEC_N = 16;         // MMA N: query heads of the group, zero-padded
+constexpr int DEC_THREADS = 192;
+
 template <int D, int G>
 struct DecCfg {
     static_assert(D == 64 || D == 128, "head size 64 or 128");
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per key/value head: 1, 2, 4 or 8");
-    static constexpr int BOXES = D / BOX_COLS;
-    static constexpr int BOX_BYTES_T = DEC_TK * 128;          // one [64 rows x 64 cols] bf16 box
-    static constexpr int TILE_BYTES = DEC_TK * D * 2;
-    static constexpr int NCH = D / 8;                         // 16-byte chunks per row
-    static constexpr int SUBS = DEC_THREADS / NCH;            // key subsets in the P V product
-    static constexpr int KPS = DEC_TK / SUBS;                 // keys per subset
-    static constexpr int K_OFF = 0;                           // + s * TILE_BYTES
-    static constexpr int V_OFF = DEC_NST * TILE_BYTES;        // + s * TILE_BYTES
-    static constexpr int Q_OFF = 2 * DEC_NST * TILE_BYTES;    // fp32 [G][D]
-    static constexpr int SC_OFF = Q_OFF + G * D * 4;          // fp32 [DEC_TK][G]: scores, then P
-    static constexpr int AL_OFF = SC_OFF + DEC_TK * G * 4;    // fp32 [G]: this tile's rescale factors
-    static constexpr int BAR_OFF = (AL_OFF + 8 * 4 + 7) / 8 * 8;  // full[NST]
-    static constexpr int MISC_OFF = BAR_OFF + DEC_NST * 8;
-    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-    // the end-of-split reduction of the P V partial sums reuses the K/V ring
-    static_assert((DEC_THREADS / 32) * G * D * 4 <= 2 * DEC_NST * TILE_BYTES, "reduction buffer");
-    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr int BOXES = D / BOX_COLS;                // 64-column boxes per row
+    static constexpr int BOX_BYTES_T = DEC_TK * 128;          // [128 slots x 64 cols] bf16
+    static constexpr int TILE_BYTES = BOXES * BOX_BYTES_T;    // one K or V tile
+    static constexpr int NST = 3 * 128 / D;                   // ring stages (each one K or one V tile)
+    static constexpr int OPB_BOX = DEC_N * 128;               // 16 rows x 64 elements, 128-byte swizzle
+    static constexpr int OPB_BYTES = 2 * OPB_BOX;             // 16 rows x 128 elements (P^T)
+    static constexpr int Q_BYTES = BOXES * OPB_BOX;           // 16 rows x D elements (q)
+    static constexpr int RING_OFF = 0;
+    static constexpr int Q_OFF = NST * TILE_BYTES;            // q, the B operand of S^T
+    static constexpr int P_OFF = Q_OFF + Q_BYTES;             // two P^T buffers
+    static constexpr int RED_OFF = P_OFF + 2 * OPB_BYTES;     // fp32 [3][4 warps][8]
+    static constexpr int BAR_OFF = RED_OFF + 3 * 4 * 8 * 4;
+    // full[NST], empty[NST], s_full[2], s_free[2], p_full[2], pv_done[2], mma_drain
+    static constexpr int NBAR = 2 * NST + 9;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;       // TMEM base (4 B), abort flag (4 B)
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack to align the base to 1 KB
+    static constexpr uint32_t TMEM_COLS = 64;
+    static constexpr uint32_t S_COL = 0;                      // + 16 * buffer
+    static constexpr uint32_t O_COL = 32;
+    static_assert(Q_OFF % 1024 == 0 && P_OFF % 1024 == 0 && OPB_BYTES % 1024 == 0, "operand alignment");
+    static_assert(NST * TILE_BYTES == 3 * 32768, "ring of 96 KB");
+    static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 };
 
-// bf16 pair (low half first) -> two fp32 values, exactly.
-__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w)
-{
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-
 template <int D, int G>
-__global__ void __launch_bounds__(DEC_THREADS)
+__global__ void __launch_bounds__(DEC_THREADS, 2)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const DecodeParams p)
+                          const DecodeParams p)
 {
     using C = DecCfg<D, G>;
+    constexpr int NST = C::NST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - raw);
-    float *const q_s = reinterpret_cast<float *>(base_ptr + C::Q_OFF);
-    float *const sc = reinterpret_cast<float *>(base_ptr + C::SC_OFF);
-    float *const alpha_s = reinterpret_cast<float *>(base_ptr + C::AL_OFF);
-    auto sK = [&](int s) { return base + C::K_OFF + s * C::TILE_BYTES; };
-    auto sV = [&](int s) { return base + C::V_OFF + s * C::TILE_BYTES; };
-    auto full = [&](int s) { return base + C::BAR_OFF + 8u * s; };
-    volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF);
+    auto ring = [&](int st) { return base + C::RING_OFF + st * C::TILE_BYTES; };
+    const uint32_t sQ = base + C::Q_OFF;
+    auto sP = [&](int pb) { return base + C::P_OFF + pb * C::OPB_BYTES; };
+    float *const red = reinterpret_cast<float *>(base_ptr + C::RED_OFF);
+    const uint32_t bars = base + C::BAR_OFF;
+    auto full = [&](int st) { return bars + 8u * st; };
+    auto empty = [&](int st) { return bars + 8u * (NST + st); };
+    auto s_full = [&](int sb) { return bars + 8u * (2 * NST + sb); };
+    auto s_free = [&](int sb) { return bars + 8u * (2 * NST + 2 + sb); };
+    auto p_full = [&](int pb) { return bars + 8u * (2 * NST + 4 + pb); };
+    auto pv_done = [&](int pb) { return bars + 8u * (2 * NST + 6 + pb); };
+    const uint32_t mma_drain = bars + 8u * (2 * NST + 8);
+    uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
+    volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
-    const int t = threadIdx.x;
+    const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x / 32), 0);
+    const int lane = static_cast<int>(threadIdx.x % 32);
     const int split = blockIdx.x;
     const int bkv = blockIdx.y;                 // b * Hkv + kv head
     const int b = bkv / p.Hkv;
@@ -103,200 +130,277 @@ __global__ void __launch_bounds__(DEC_THREADS)
 
     if (ntiles == 0) {
         // no cached slot in this split: an empty partial (max -inf, sum 0)
-        for (int i = t; i < G * (D + 2); i += DEC_THREADS) {
+        for (int i = threadIdx.x; i < G * (D + 2); i += DEC_THREADS) {
             const int g = i / (D + 2), c = i % (D + 2);
             part[(prow + g) * (D + 2) + c] = (c == D) ? -CUDART_INF_F : 0.f;
         }
         return;
     }
 
-    if (t == 0) {
-        for (int s = 0; s < DEC_NST; ++s) mbar_init(full(s), 1);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < NST; ++st) {
+            mbar_init(full(st), 1);
+            mbar_init(empty(st), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_full(i), 1);
+            mbar_init(s_free(i), 4 * 32);
+            mbar_init(p_full(i), 4 * 32);
+            mbar_init(pv_done(i), 1);
+        }
+        mbar_init(mma_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // the group's query rows, fp32
-    for (int i = t; i < G * D; i += DEC_THREADS)
-        q_s[i] = __bfloat162float(p.q[(static_cast<size_t>(b) * p.H + h0) * D + i]);
+    // q of the group's G heads as a 16-row K-major operand (128-byte swizzle:
+    // 16-byte chunk j of row g at chunk j ^ (g % 8)); rows >= G and both P^T
+    // buffers zero (rows >= G of P^T stay zero for good).
+    for (int i = threadIdx.x; i < DEC_N * (D / 8); i += DEC_THREADS) {
+        const int g = i / (D / 8), j = i % (D / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (g < G)
+            v = *reinterpret_cast<const uint4 *>(p.q + (static_cast<size_t>(b) * p.H + h0 + g) * D + 8 * j);
+        const uint32_t addr = sQ + (j / 8) * C::OPB_BOX + g * 128 +
+                              ((static_cast<uint32_t>(j % 8) ^ static_cast<uint32_t>(g & 7)) * 16);
+        st_shared_v4(addr, v.x, v.y, v.z, v.w);
+    }
+    for (int i = threadIdx.x; i < 2 * C::OPB_BYTES / 16; i += DEC_THREADS)
+        st_shared_v4(sP(0) + i * 16, 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     const Waiter wt{abort_flag, p.status};
 
-    auto issue = [&](int tile) {
-        const int s = tile % DEC_NST;
-        mbar_arrive_expect_tx(full(s), 2 * C::TILE_BYTES);
-        const int slot = s0 + tile * DEC_TK;
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        const uint32_t leader = elect_one();
+        const int nitems = 2 * ntiles;  // item 2i: K_i, item 2i + 1: V_i
+        int issued = 0;
+        for (; issued < nitems; ++issued) {
+            const int st = issued % NST;
+            if (issued >= NST &&
+                !__all_sync(0xffffffffu, wt.wait(empty(st), ((issued / NST) - 1) & 1u)))
+                break;
+            const int slot = s0 + (issued / 2) * DEC_TK;
+            const CUtensorMap *map = (issued & 1) ? &tmV : &tmK;
+            mbar_arrive_expect_tx_if(leader, full(st), C::TILE_BYTES);
 #pragma unroll
-        for (int bx = 0; bx < C::BOXES; ++bx) {
-            tma_load_3d(sK(s) + bx * C::BOX_BYTES_T, &tmK, full(s), bx * BOX_COLS, slot, bkv);
-            tma_load_3d(sV(s) + bx * C::BOX_BYTES_T, &tmV, full(s), bx * BOX_COLS, slot, bkv);
+            for (int bx = 0; bx < C::BOXES; ++bx)
+                tma_load_3d_if(leader, ring(st) + bx * C::BOX_BYTES_T, map, full(st), bx * BOX_COLS, slot, bkv);
         }
-    };
-    int issued = 0;  // tiles whose loads thread 0 has issued
-    if (t == 0) {
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
-        for (; issued < DEC_NST && issued < ntiles; ++issued) issue(issued);
-    }
-
-    // running max (log2 units) and sum of query head g, held by every lane of
-    // warp g (warps g >= G leave them unused)
-    float m_run = -CUDART_INF_F, l_run = 0.f;
-    // P V accumulators: 8 columns [8c, 8c + 8) of every head, over this
-    // thread's key subset of each tile
-    const int pc = t % C::NCH;
-    const int psub = t / C::NCH;
-    float acc[G][8];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-
-    bool ok = true;
-    for (int tile = 0; tile < ntiles; ++tile) {
-        const int s = tile % DEC_NST;
-        ok = __syncthreads_and(wt.wait(full(s), (tile / DEC_NST) & 1u));
-        if (!ok) break;
-        const int slot0 = s0 + tile * DEC_TK;
-        // ---- scores: thread = key k, heads g = gq, gq + 4, ...
-        {
-            const int k = t % DEC_TK;
-            const int gq = t / DEC_TK;
-            if (gq < G) {
-                constexpr int GPT = (G + 3) / 4;  // heads per thread
-                float dot[GPT];
-#pragma unroll
-                for (int i = 0; i < GPT; ++i) dot[i] = 0.f;
-#pragma unroll 4
-                for (int j = 0; j < C::NCH; ++j) {
-                    const uint32_t addr = sK(s) + (j / 8) * C::BOX_BYTES_T + k * 128 +
-                                          ((static_cast<uint32_t>(j % 8) ^ static_cast<uint32_t>(k & 7)) * 16);
-                    uint4 kw;
-                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(kw.x), "=r"(kw.y), "=r"(kw.z), "=r"(kw.w)
-                                 : "r"(addr));
-                    const float2 k01 = bf16x2_to_f2(kw.x), k23 = bf16x2_to_f2(kw.y);
-                    const float2 k45 = bf16x2_to_f2(kw.z), k67 = bf16x2_to_f2(kw.w);
-#pragma unroll
-                    for (int i = 0; i < GPT; ++i) {
-                        const int g = gq + 4 * i;
-                        if (g < G) {
-                            const float4 qa = *reinterpret_cast<const float4 *>(q_s + g * D + 8 * j);
-                            const float4 qb = *reinterpret_cast<const float4 *>(q_s + g * D + 8 * j + 4);
-                            float2 d2 = ffma2(k01, make_float2(qa.x, qa.y), make_float2(dot[i], 0.f));
-                            d2 = ffma2(k23, make_float2(qa.z, qa.w), d2);
-                            d2 = ffma2(k45, make_float2(qb.x, qb.y), d2);
-                            d2 = ffma2(k67, make_float2(qb.z, qb.w), d2);
-                            dot[i] = d2.x + d2.y;
-                        }
-                    }
-                }
-                const bool valid = slot0 + k < s1;
-#pragma unroll
-                for (int i = 0; i < GPT; ++i) {
-                    const int g = gq + 4 * i;
-                    if (g < G) sc[k * G + g] = valid ? dot[i] * p.scale_log2 : -CUDART_INF_F;
-                }
+        // copies still in flight must land before the CTA exits
+        for (int st = 0; st < NST; ++st) {
+            if (issued > st) {
+                const int last = st + ((issued - 1 - st) / NST) * NST;
+                wt.drain(full(st), (last / NST) & 1u);
             }
         }
-        __syncthreads();
-        // ---- online softmax: warp g handles head g over the tile's keys
-        {
-            const int w = t / 32, lane = t % 32;
-            if (w < G) {
-                const float a = sc[lane * G + w], c = sc[(lane + 32) * G + w];
-                float mx = fmaxf(a, c);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t leader = elect_one();
+        constexpr uint32_t idesc_s = idesc_bf16_f32(DEC_TK, DEC_N, 0, 0);  // K, q both K-major
+        constexpr uint32_t idesc_o = idesc_bf16_f32(D, DEC_N, 1, 0);       // V^T MN-major, P^T K-major
+        const uint64_t qdesc = smem_desc_sw128(sQ, 16, 1024);
+        // S(i) = K_i q^T into S buffer i % 2
+        auto issue_s = [&](int i) -> bool {
+            const int item = 2 * i, st = item % NST;
+            if (!__all_sync(0xffffffffu, wt.wait(full(st), (item / NST) & 1u))) return false;
+            // the softmax must have read S(i - 2) out of this buffer
+            if (i >= 2 && !__all_sync(0xffffffffu, wt.wait(s_free(i % 2), ((i - 2) / 2) & 1u))) return false;
+            tc_fence_after();
+            const uint64_t kdesc = smem_desc_sw128(ring(st), 16, 1024);
+            const uint32_t d_col = tmem + C::S_COL + DEC_N * (i % 2);
 #pragma unroll
-                for (int o = 16; o >= 1; o /= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                const float m_new = fmaxf(m_run, mx);  // finite: the first key of a tile is valid
-                const float pa = ex2_approx(a - m_new), pc2 = ex2_approx(c - m_new);
-                sc[lane * G + w] = pa;
-                sc[(lane + 32) * G + w] = pc2;
-                float sum = pa + pc2;
-#pragma unroll
-                for (int o = 16; o >= 1; o /= 2) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                const float alpha = ex2_approx(m_run - m_new);  // 0 on the first tile
-                l_run = l_run * alpha + sum;
-                m_run = m_new;
-                if (lane == 0) alpha_s[w] = alpha;
+            for (int k = 0; k < D / 16; ++k) {
+                const uint64_t koff = static_cast<uint64_t>(((k / 4) * C::BOX_BYTES_T + (k % 4) * 32) >> 4);
+                const uint64_t qoff = static_cast<uint64_t>(((k / 4) * C::OPB_BOX + (k % 4) * 32) >> 4);
+                mma_bf16_ss_if(leader, d_col, kdesc + koff, qdesc + qoff, idesc_s, k > 0 ? 1u : 0u);
             }
+            mma_commit_if(leader, s_full(i % 2));
+            mma_commit_if(leader, empty(st));
+            return true;
+        };
+        // O^T += V_i^T P_i^T
+        auto issue_pv = [&](int i) -> bool {
+            const int item = 2 * i + 1, st = item % NST;
+            if (!__all_sync(0xffffffffu, wt.wait(full(st), (item / NST) & 1u))) return false;
+            if (!__all_sync(0xffffffffu, wt.wait(p_full(i % 2), (i / 2) & 1u))) return false;
+            tc_fence_after();
+            const uint64_t vdesc = smem_desc_sw128(ring(st), C::BOX_BYTES_T, 1024);
+            const uint64_t pdesc = smem_desc_sw128(sP(i % 2), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < DEC_TK / 16; ++k) {
+                const uint64_t poff = static_cast<uint64_t>(((k / 4) * C::OPB_BOX + (k % 4) * 32) >> 4);
+                mma_bf16_ss_if(leader, tmem + C::O_COL, vdesc + static_cast<uint64_t>(k * 128), pdesc + poff,
+                               idesc_o, (i > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit_if(leader, pv_done(i % 2));
+            mma_commit_if(leader, empty(st));
+            return true;
+        };
+        bool ok = issue_s(0);
+        for (int i = 0; ok && i < ntiles; ++i) {
+            if (i + 1 < ntiles) ok = issue_s(i + 1);
+            if (ok) ok = issue_pv(i);
         }
-        __syncthreads();
-        // ---- O += P V over this thread's keys, all heads, columns [8 pc, 8 pc + 8)
-        {
-            float al[G];
+        // every MMA this warp issued must finish before TMEM is freed
+        mma_commit_if(leader, mma_drain);
+        wt.drain(mma_drain, 0);
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int sw = warp % 4;                    // TMEM subpartition of this warp
+        const int r = sw * 32 + lane;               // slot in the tile (= TMEM lane)
+        // column of d that O^T holds in this thread's lane (d = 64: lanes
+        // 16-31 of each quarter hold none)
+        const int dcol = (D == 128) ? r : 16 * sw + lane;
+        const bool has_dcol = (D == 128) || lane < 16;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(sw * 32) << 16);
+        const float sc = p.scale_log2;
+        float m_run[G], l_part[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) al[g] = alpha_s[g];
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[g][e] *= al[g];
-#pragma unroll
-            for (int kk = 0; kk < C::KPS; ++kk) {
-                const int k = psub * C::KPS + kk;
-                // slots past the cache: P is 0, but the slot may hold NaN
-                // (0 * NaN would reach O), so it is skipped
-                if (slot0 + k >= s1) continue;
-                const uint32_t addr = sV(s) + (pc / 8) * C::BOX_BYTES_T + k * 128 +
-                                      ((static_cast<uint32_t>(pc % 8) ^ static_cast<uint32_t>(k & 7)) * 16);
-                uint4 vw;
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(vw.x), "=r"(vw.y), "=r"(vw.z), "=r"(vw.w)
-                             : "r"(addr));
-                const float2 v01 = bf16x2_to_f2(vw.x), v23 = bf16x2_to_f2(vw.y);
-                const float2 v45 = bf16x2_to_f2(vw.z), v67 = bf16x2_to_f2(vw.w);
+        for (int g = 0; g < G; ++g) {
+            m_run[g] = -CUDART_INF_F;
+            l_part[g] = 0.f;
+        }
+        // Every tile the four warps agree (bar.red.and) before they exchange
+        // maxima, so a wait that gives up in one warp ends the loop in all.
+        bool ok = true;
+        for (int i = 0; i < ntiles; ++i) {
+            const int sb = i % 2;
+            bool okw = __all_sync(0xffffffffu, wt.wait(s_full(sb), (i / 2) & 1u));
+            float s[G];
+            if (okw) {
+                tc_fence_after();
+                uint32_t sv[8];
+                tmem_ld8(lane_base + C::S_COL + DEC_N * sb, sv);
+                tc_fence_before();
+                mbar_arrive(s_free(sb));
+                const bool valid = s0 + i * DEC_TK + r < s1;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float pw = sc[k * G + g];
-                    const float2 p2 = make_float2(pw, pw);
-                    float2 r01 = ffma2(v01, p2, make_float2(acc[g][0], acc[g][1]));
-                    float2 r23 = ffma2(v23, p2, make_float2(acc[g][2], acc[g][3]));
-                    float2 r45 = ffma2(v45, p2, make_float2(acc[g][4], acc[g][5]));
-                    float2 r67 = ffma2(v67, p2, make_float2(acc[g][6], acc[g][7]));
-                    acc[g][0] = r01.x; acc[g][1] = r01.y; acc[g][2] = r23.x; acc[g][3] = r23.y;
-                    acc[g][4] = r45.x; acc[g][5] = r45.y; acc[g][6] = r67.x; acc[g][7] = r67.y;
+                    s[g] = valid ? __uint_as_float(sv[g]) * sc : -CUDART_INF_F;
+                    float mx = s[g];
+#pragma unroll
+                    for (int o = 16; o >= 1; o /= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    if (lane == 0) red[(sb * 4 + sw) * 8 + g] = mx;
+                }
+            }
+            ok = named_bar_and(1, 4 * 32, okw);
+            if (!ok) break;
+            const int slot0 = s0 + i * DEC_TK;
+            const bool valid = slot0 + r < s1;
+            float alpha[G], pr[G];
+            bool grew = false;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float tmax = fmaxf(fmaxf(red[(sb * 4 + 0) * 8 + g], red[(sb * 4 + 1) * 8 + g]),
+                                         fmaxf(red[(sb * 4 + 2) * 8 + g], red[(sb * 4 + 3) * 8 + g]));
+                const float m_new = fmaxf(m_run[g], tmax);  // finite: a tile's first slot is valid
+                grew = grew || (m_new > m_run[g]);
+                alpha[g] = ex2_approx(m_run[g] - m_new);    // 0 on the first tile
+                pr[g] = ex2_approx(s[g] - m_new);           // 0 for slots past the cache
+                l_part[g] = fmaf(l_part[g], alpha[g], pr[g]);
+                m_run[g] = m_new;
+            }
+            // P^T buffer sb was last read by PV(i - 2)
+            if (i >= 2) okw = __all_sync(0xffffffffu, wt.wait(pv_done(sb), ((i - 2) / 2) & 1u));
+            // O^T must be rescaled when a head's max grew: it holds the tiles
+            // before i once PV(i - 1) is done (the decision is the same in
+            // every thread: all read the same maxima)
+            if (okw && i > 0 && grew) {
+                okw = __all_sync(0xffffffffu, wt.wait(pv_done((i - 1) % 2), ((i - 1) / 2) & 1u));
+                if (okw) {
+                    tc_fence_after();
+                    uint32_t o[8];
+                    tmem_ld8(lane_base + C::O_COL, o);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+                    tmem_st8(lane_base + C::O_COL, o);
+                    tmem_wait_st();
+                }
+            }
+            // Slots in [L, W) hold whatever the caller left there; their P is
+            // 0, but 0 * NaN would still reach O, so their V rows are zeroed
+            // (slots >= W already read as zero).
+            if (okw && slot0 + DEC_TK > s1 && s1 < p.W) {
+                const int item = 2 * i + 1, st = item % NST;
+                okw = __all_sync(0xffffffffu, wt.wait(full(st), (item / NST) & 1u));
+                if (okw && !valid && slot0 + r < p.W) {
+#pragma unroll
+                    for (int bx = 0; bx < C::BOXES; ++bx)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            st_shared_v4(ring(st) + bx * C::BOX_BYTES_T + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+                }
+            }
+            if (okw) {
+                // P^T: row g (head), column r (slot)
+                const uint32_t col = sP(sb) + (r / 64) * C::OPB_BOX +
+                                     ((static_cast<uint32_t>((r % 64) / 8)) * 16) + (r % 8) * 2;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const uint32_t addr = (col + g * 128) ^ (static_cast<uint32_t>(g & 7) << 4);
+                    const unsigned short h = __bfloat16_as_ushort(__float2bfloat16_rn(pr[g]));
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(h) : "memory");
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full(sb));
+            }
+            ok = okw;
+        }
+        // the four warps agree on how the loop ended
+        ok = named_bar_and(1, 4 * 32, ok);
+        bool okw = ok;
+        if (ok) {
+            const int last = ntiles - 1;
+            okw = __all_sync(0xffffffffu, wt.wait(pv_done(last % 2), (last / 2) & 1u));
+            if (okw) {
+                tc_fence_after();
+                uint32_t o[8];
+                tmem_ld8(lane_base + C::O_COL, o);
+                // O^T: this lane holds column dcol of d, TMEM column g = head g
+                if (has_dcol) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) part[(prow + g) * (D + 2) + dcol] = __uint_as_float(o[g]);
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float sum = l_part[g];
+#pragma unroll
+                for (int o = 16; o >= 1; o /= 2) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane == 0) red[(2 * 4 + sw) * 8 + g] = sum;
+            }
+        }
+        ok = named_bar_and(1, 4 * 32, okw);
+        if (ok) {
+            // this split's max and sum of head g, written by thread g (every
+            // thread holds the same running maxima)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                if (r == g) {
+                    const float l = (red[(2 * 4 + 0) * 8 + g] + red[(2 * 4 + 1) * 8 + g]) +
+                                    (red[(2 * 4 + 2) * 8 + g] + red[(2 * 4 + 3) * 8 + g]);
+                    part[(prow + g) * (D + 2) + D] = m_run[g];
+                    part[(prow + g) * (D + 2) + D + 1] = l;
                 }
             }
         }
-        // every thread is done with this stage's K and V (and with sc and
-        // alpha_s, which the next tile rewrites): refill the stage
-        __syncthreads();
-        if (t == 0 && issued < ntiles) issue(issued++);
     }
-    // copies still in flight must land before the CTA exits
-    if (t == 0)
-        for (int s = 0; s < DEC_NST; ++s)
-            if (issued > s) wt.drain(full(s), ((issued - 1 - s) / DEC_NST) & 1u);
-    if (!__syncthreads_and(ok)) return;
 
-    // ---- reduce the P V partial sums over key subsets: lanes t and t ^ NCH
-    // share a column chunk within a warp (for D = 128; D = 64 has more
-    // subsets per warp), then the warps through shared memory
-    float *const red = reinterpret_cast<float *>(base_ptr + C::K_OFF);  // ring is idle now
-#pragma unroll
-    for (int o = C::NCH; o < 32; o *= 2)
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
-    const int w = t / 32, lane = t % 32;
-    if (lane < C::NCH) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) red[(w * G + g) * D + 8 * pc + e] = acc[g][e];
-    }
-    if (w < G && lane == 0) {
-        // this split's max and sum of head w
-        part[(prow + w) * (D + 2) + D] = m_run;
-        part[(prow + w) * (D + 2) + D + 1] = l_run;
-    }
+    tc_fence_before();
     __syncthreads();
-    for (int i = t; i < G * D; i += DEC_THREADS) {
-        const int g = i / D, c = i % D;
-        float s = 0.f;
-#pragma unroll
-        for (int ww = 0; ww < DEC_THREADS / 32; ++ww) s += red[(ww * G + g) * D + c];
-        part[(prow + g) * (D + 2) + c] = s;
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 

@@ -298,12 +298,11 @@ ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
  *
  * A negative pos[b] is read as 0. Slots no cached position occupies yet
  * (slot >= pos[b] + 1 while pos[b] < W - 1) may hold any bits, NaN included:
- * they never reach the result. Arithmetic: d = 128 on the tensor cores
- * (bf16 products, fp32 scores and accumulation, softmax weights rounded to
- * bf16 for the value product, as in attn_fwd); d = 64 on the CUDA cores in
- * fp32 throughout. O is rounded to bf16. Two kernels are enqueued: per
- * (split of the slots, sequence, kv head) partial results, then their
- * log-sum-exp merge. Returns as attn_fwd.
+ * they never reach the result. Arithmetic: tensor cores (bf16 products,
+ * fp32 scores and accumulation, softmax weights rounded to bf16 for the
+ * value product, as in attn_fwd); O is rounded to bf16. Two kernels are
+ * enqueued: per (split of the slots, sequence, kv head) partial results,
+ * then their log-sum-exp merge. Returns as attn_fwd.
  */
 ATTN_API int attn_decode(const void *q, const void *k_cache, const void *v_cache, const int *pos,
                          void *o, float *lse, void *workspace, size_t workspace_bytes, int B,

@@ -188,11 +188,19 @@ def test_attn_decode_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
 
 
 def test_decode_workspace_size(attn):
-    # per-split partials: nsplit * B * H * (d + 2) fp32, nsplit from the split rule
+    # per-split partials: nsplit * B * H * (d + 2) fp32; the split rule cuts
+    # the 128-slot tiles into splits minimising waves x (tiles per split + 1)
+    # over 2 x 148 resident CTAs (first minimum, 1 to 64 splits)
     def expect(B, H, Hkv, W, d):
-        tiles = (W + 63) // 64
-        ns = max(1, min(tiles, (4 * 148 + B * Hkv - 1) // (B * Hkv)))
-        chunk = ((tiles + ns - 1) // ns) * 64
+        tiles = (W + 127) // 128
+        best = None
+        for ns in range(1, min(tiles, 64) + 1):
+            per = (tiles + ns - 1) // ns
+            ctas = B * Hkv * ((tiles + per - 1) // per)
+            cost = ((ctas + 295) // 296) * (per + 1)
+            if best is None or cost < best[0]:
+                best = (cost, per)
+        chunk = best[1] * 128
         return ((W + chunk - 1) // chunk) * B * H * (d + 2) * 4
     for shape in [(1, 1, 1, 1, 64), (2, 8, 2, 4096, 128), (64, 32, 8, 4096, 128), (3, 4, 4, 200, 64)]:
         assert attn.decode_workspace_bytes(*shape) == expect(*shape)
