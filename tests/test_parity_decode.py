@@ -1,9 +1,10 @@
 """Decode against rolling caches (through the C ABI) against the fp64 oracle.
 
 Small problems cover every grouped-query ratio, head size, partially filled
-and wrapped caches, cache sizes that are not a multiple of the 64- or
-128-slot tile (head size 64 and 128 run different kernels), mixed positions
-within a batch, and caches whose unused slots hold NaN; the full-size
+and wrapped caches, cache sizes around multiples of the kernel's 128-slot
+tile, mixed positions within a batch, splits of the slots that lie wholly
+or partly past the cached positions, and caches whose unused slots hold
+NaN; the full-size
 workload (64 sequences at position 32767 against 4096-slot caches) is
 compared on every row.
 """
