@@ -63,10 +63,13 @@ constexpr int STATUS_WAIT_TIMEOUT = 1;
 // dominant term: too much for peaked rows.)
 
 // Exponentials computed on the FMA pipe instead of the MUFU unit: out of every
-// 16 pairs of a row, ATTN_EX2_EMU_D* pairs (spread evenly: pair i when
-// i * EMU mod 16 < EMU) use the polynomial.
+// 16 pairs of a row, ATTN_EX2_EMU_D* pairs use the polynomial (at d = 128
+// spread evenly, pair i when i * EMU mod 16 < EMU; at d = 64 the first ones).
+// The splits and the row-max form per head size are the fastest measured in
+// runs long enough to reach the power cap: at d = 64 more FMA-pipe work
+// gains per clock but lowers the clock more.
 #ifndef ATTN_EX2_EMU_D64
-#define ATTN_EX2_EMU_D64 4
+#define ATTN_EX2_EMU_D64 3
 #endif
 #ifndef ATTN_EX2_EMU_D128
 #define ATTN_EX2_EMU_D128 5
@@ -118,6 +121,8 @@ struct FwdCfg {
     static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER == THREADS * REGS_LAUNCH,
                   "register split must use exactly the launch allocation");
     static constexpr int EX2_EMU = (D == 128) ? ATTN_EX2_EMU_D128 : ATTN_EX2_EMU_D64;
+    static constexpr bool EMU_SPREAD = (D == 128);  // polynomial pairs spread along the row
+    static constexpr bool MAX3 = (D == 128);        // row max with three-input max
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -545,17 +550,30 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 for (int c = 0; c < BN; ++c)
                     if (c > hi || c < lo) sv[c] = f2u(-CUDART_INF_F);
             }
-            // row max: eight running maxima of three-input max instructions
+            // row max: eight running maxima, of three-input max instructions
+            // at d = 128 and of two-input ones at d = 64 (the faster form of
+            // each under the power cap)
             float pm[8];
+            if constexpr (C::MAX3) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = fmax3(u2f(sv[i]), u2f(sv[8 + i]), u2f(sv[16 + i]));
+                for (int i = 0; i < 8; ++i) pm[i] = fmax3(u2f(sv[i]), u2f(sv[8 + i]), u2f(sv[16 + i]));
 #pragma unroll
-            for (int c = 24; c + 16 <= BN; c += 16)
+                for (int c = 24; c + 16 <= BN; c += 16)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], u2f(sv[c + i]), u2f(sv[c + 8 + i]));
+                    for (int i = 0; i < 8; ++i) pm[i] = fmax3(pm[i], u2f(sv[c + i]), u2f(sv[c + 8 + i]));
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], u2f(sv[BN - 8 + i]));
-            const float tmax = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+                for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], u2f(sv[BN - 8 + i]));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pm[i] = fmaxf(u2f(sv[i]), u2f(sv[8 + i]));
+#pragma unroll
+                for (int c = 16; c < BN; c += 8)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) pm[i] = fmaxf(pm[i], u2f(sv[c + i]));
+            }
+            const float tmax = C::MAX3 ? fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]))
+                                       : fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             const float mnew = fmaxf(mx, tmax * sc);
             const bool rescale = mnew > mx;
             // alpha = 2^(m_old - m_new): 1 when the max did not grow, 0 when
@@ -580,8 +598,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
                     float e0, e1;
                     if constexpr (EMU > 0) {
-                        // EMU of every 16 pairs, spread evenly along the row
-                        if (((i * EMU) % 16) < EMU) {
+                        // EMU of every 16 pairs: spread evenly along the
+                        // row, or the first EMU of each 16
+                        if ((C::EMU_SPREAD ? ((i * EMU) % 16) : (i % 16)) < EMU) {
                             ex2_poly_x2(x.x, x.y, e0, e1);
                         } else {
                             e0 = ex2_approx(x.x);
