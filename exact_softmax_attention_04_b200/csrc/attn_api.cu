@@ -98,6 +98,37 @@ struct Staging {
 };
 Staging g_staging[kMaxDevices];
 
+// Side streams of attn_fwd_host, one per copy direction, so that one chunk
+// of heads is copied in while another is computed and a third copied out.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t entry = nullptr, done = nullptr;
+    cudaEvent_t in[kHostChunks] = {}, ran[kHostChunks] = {};
+    bool ready = false;
+};
+HostPipe g_pipe[kMaxDevices];
+
+// The current device's streams and events, created on first use (caller
+// holds g_mu).
+int host_pipe(int dev, HostPipe **out)
+{
+    HostPipe &hp = g_pipe[dev];
+    if (!hp.ready) {
+        bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+        for (int c = 0; ok && c < kHostChunks; ++c)
+            ok = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&hp.ran[c], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return ATTN_ERR_CUDA;  // what was created is kept and reused next time
+        hp.ready = true;
+    }
+    *out = &hp;
+    return ATTN_OK;
+}
+
 int check_args(const void *q, const void *k, const void *v, const void *o, const void *lse, int B,
                int H, int n, int d, float scale, int causal, int window, bool device_buffers,
                int Hkv = -1)
@@ -265,15 +296,62 @@ extern "C" int attn_fwd_host(const void *q, const void *k, const void *v, void *
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *dq = buf, *dk = buf + tb, *dv = buf + 2 * tb, *dout = buf + 3 * tb;
     float *dl = reinterpret_cast<float *>(buf + 4 * tb);
-    if (cudaMemcpyAsync(dq, q, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    rc = attn_fwd(dq, dk, dv, dout, dl, B, H, n, d, scale, causal, window, stream);
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
+               *hv = static_cast<const char *>(v);
+    char *ho = static_cast<char *>(o);
+
+    // Heads are independent: cut them into up to kHostChunks chunks and
+    // pipeline them (copy-in on one side stream, kernel on `stream`, copy-out
+    // on the other), unless the problem is small enough for one pass.
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    const size_t head_bytes = static_cast<size_t>(n) * d * 2;
+    int chunks = (3 * elems * 2 >= (static_cast<size_t>(16) << 20)) ? kHostChunks : 1;
+    if (chunks > bh) chunks = static_cast<int>(bh);
+    const int64_t per = (bh + chunks - 1) / chunks;
+    chunks = static_cast<int>((bh + per - 1) / per);
+    if (chunks == 1) {
+        if (cudaMemcpyAsync(dq, q, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync(dk, k, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+            cudaMemcpyAsync(dv, v, elems * 2, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        rc = attn_fwd(dq, dk, dv, dout, dl, B, H, n, d, scale, causal, window, stream);
+        if (rc != ATTN_OK) return rc;
+        if (cudaMemcpyAsync(o, dout, elems * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+            cudaMemcpyAsync(lse, dl, static_cast<size_t>(B) * H * n * 4, cudaMemcpyDeviceToHost, st) !=
+                cudaSuccess)
+            return ATTN_ERR_CUDA;
+        return ATTN_OK;
+    }
+    HostPipe *hp = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        rc = host_pipe(dev, &hp);
+    }
     if (rc != ATTN_OK) return rc;
-    if (cudaMemcpyAsync(o, dout, elems * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(lse, dl, static_cast<size_t>(B) * H * n * 4, cudaMemcpyDeviceToHost, st) !=
-            cudaSuccess)
+    // Side-stream work starts after everything already on `stream` (the
+    // staging buffers may still be in use by an earlier call), and `stream`
+    // continues only once the last copy-out is done.
+    if (cudaEventRecord(hp->entry, st) != cudaSuccess || cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    for (int c = 0; c < chunks; ++c) {
+        const int64_t h0 = c * per;
+        const int hc = static_cast<int>(bh - h0 < per ? bh - h0 : per);
+        const size_t off = static_cast<size_t>(h0) * head_bytes, bytes = static_cast<size_t>(hc) * head_bytes;
+        const size_t loff = static_cast<size_t>(h0) * n, lbytes = static_cast<size_t>(hc) * n * 4;
+        if (cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+            cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+            cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+            cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp->in[c], 0) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        rc = attn_fwd(dq + off, dk + off, dv + off, dout + off, dl + loff, 1, hc, n, d, scale, causal, window,
+                      stream);
+        if (rc != ATTN_OK) return rc;
+        if (cudaEventRecord(hp->ran[c], st) != cudaSuccess || cudaStreamWaitEvent(hp->d2h, hp->ran[c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(ho + off, dout + off, bytes, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess ||
+            cudaMemcpyAsync(lse + loff, dl + loff, lbytes, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+    }
+    if (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp->done, 0) != cudaSuccess)
         return ATTN_ERR_CUDA;
     return ATTN_OK;
 }

@@ -138,12 +138,19 @@ ATTN_API int attn_fwd_blocklocal(const void *q, const void *k, const void *v, vo
  *   q, k, v : host, bf16 [B, H, n, d] (pinned memory makes the copies async)
  *   o, lse  : host, written (bf16 [B, H, n, d] and fp32 [B, H, n])
  *
- * Enqueues on `stream`: host-to-device copies of q, k, v into library-owned
- * staging buffers, attn_fwd, and device-to-host copies of o and lse. The
- * caller synchronizes `stream` (or calls attn_sync_status) before reading o
- * and lse. Staging buffers are per device and shared by all calls: calls on
- * different streams of one device must not overlap. Returns as attn_fwd, or
- * ATTN_ERR_CUDA if growing the staging buffers fails.
+ * Enqueues host-to-device copies of q, k, v into library-owned staging
+ * buffers, attn_fwd, and device-to-host copies of o and lse. Problems of
+ * 16 MB of inputs or more are cut into up to 8 chunks of heads and
+ * pipelined: the copies run on two library-owned side streams (one per
+ * direction) and the kernels on `stream`, so one chunk is copied in while
+ * another is computed and a third is copied out. The side streams start
+ * after the work already on `stream`, and `stream` waits for the last copy,
+ * so the call is ordered on `stream` as a whole. The caller synchronizes
+ * `stream` (or calls attn_sync_status) before reading o and lse. Staging
+ * buffers and side streams are per device and shared by all calls: calls
+ * on different streams of one device must not overlap. Returns as attn_fwd,
+ * or ATTN_ERR_CUDA if growing the staging buffers or creating the side
+ * streams fails.
  */
 ATTN_API int attn_fwd_host(const void *q, const void *k, const void *v, void *o, float *lse,
                   int B, int H, int n, int d, float scale, int causal, int window,

@@ -131,6 +131,22 @@ def test_host_entry_point_matches_device_entry_point(attn):
     assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
 
 
+def test_host_entry_pipelined_chunks_equal_device(attn):
+    """Large enough for the host entry point to pipeline its copies over
+    chunks of heads (13 heads: a ragged last chunk), called twice back to
+    back into different outputs with no synchronisation in between."""
+    qa, ka, va = synth.make_qkv(1, 13, 4096, 128, seed=91)
+    qb, kb, vb = synth.make_qkv(1, 13, 4096, 128, seed=92)
+    o_a, l_a = _gpu(attn, qa, ka, va, True, 1000)
+    o_b, l_b = _gpu(attn, qb, kb, vb, True, 1000)
+    pinned = [t.pin_memory() for t in (qa, ka, va, qb, kb, vb)]
+    o1, l1 = attn.attn_fwd_host(*pinned[:3], causal=True, window=1000)
+    o2, l2 = attn.attn_fwd_host(*pinned[3:], causal=True, window=1000)
+    assert attn.sync_status() == attn.ATTN_OK
+    assert torch.equal(o1, o_a.cpu()) and torch.equal(l1, l_a.cpu())
+    assert torch.equal(o2, o_b.cpu()) and torch.equal(l2, l_b.cpu())
+
+
 @pytest.mark.parametrize("wl", synth.sweep(), ids=lambda w: w.name)
 def test_sweep_cells_sampled(attn, oracle_mod, wl):
     rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=24, bound_every=16)
