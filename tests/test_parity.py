@@ -153,6 +153,16 @@ def test_sweep_cells_sampled(attn, oracle_mod, wl):
     _sampled_check(attn, oracle_mod, wl, rows)
 
 
+@pytest.mark.parametrize("wl", [synth.Workload("B1-H2-n50001-d128-causal", 1, 2, 50001, 128, True, q_std=2.0, seed=3),
+                                synth.Workload("B1-H3-n40007-d64-window1000", 1, 3, 40007, 64, True, 1000, seed=4)],
+                         ids=lambda w: w.name)
+def test_large_ragged_lengths_sampled(attn, oracle_mod, wl):
+    """Long sequences whose length is no multiple of the 128-row tile: the
+    last, partly filled query and key tiles among the sampled rows."""
+    rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=24, bound_every=64, edge=40)
+    _sampled_check(attn, oracle_mod, wl, rows)
+
+
 @pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.CAUSAL_N131072,
                                 synth.SYM_N16384], ids=lambda w: w.name)
 def test_full_size_workloads_sampled(attn, oracle_mod, wl):
@@ -236,6 +246,24 @@ def test_block_mask_small_in_full(attn, oracle_mod, d, block, causal):
     assert attn.sync_status() == attn.ATTN_OK
     o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, sc, causal, -1, block)
     assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"block{block} d{d} c{causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_of_n_tokens_or_more_is_no_mask(attn, oracle_mod, d, causal):
+    """One block covers the sequence: the keys of attn_fwd without a window,
+    bit for bit; one token fewer leaves a second block of one token."""
+    n = 333
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=5 + d)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o0, l0 = attn.attn_fwd(qc, kc, vc, None, causal, -1)
+    for block in (n, 4 * n):
+        o, lse = attn.attn_fwd(qc, kc, vc, None, causal, -1, block=block)
+        assert torch.equal(o, o0) and torch.equal(lse, l0)
+    o, lse = attn.attn_fwd(qc, kc, vc, None, causal, -1, block=n - 1)
+    assert attn.sync_status() == attn.ATTN_OK
+    o_ref, lse_ref = oracle_mod.attn_fwd(q, k, v, 1.0 / np.sqrt(d), causal, -1, n - 1)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, f"block n-1 d{d} c{causal}")
 
 
 def test_block_mask_gqa(attn, oracle_mod):

@@ -108,7 +108,10 @@ def test_bwd_deterministic_and_dirty_workspace(attn, d):
         assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2 * a[0].float().abs().max().item()
 
 
-@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.SYM_N16384],
+@pytest.mark.parametrize("wl", [synth.FULL_N8192, synth.WINDOW_N32768, synth.SYM_N16384,
+                                # lengths that are no multiple of the 128-row tile
+                                synth.Workload("B1-H2-n20011-d128-causal", 1, 2, 20011, 128, True, q_std=2.0, seed=7),
+                                synth.Workload("B1-H2-n12345-d64-window2000", 1, 2, 12345, 64, True, 2000, seed=8)],
                          ids=lambda w: w.name)
 def test_bwd_full_size_workloads_sampled(attn, oracle_mod, wl):
     q, k, v = synth.make_inputs(wl)
