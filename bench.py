@@ -55,17 +55,42 @@ def peaks():
         return FALLBACK_BF16_TFLOPS, FALLBACK_HBM_GBS, "fallback"
 
 
-# Device code of the timed forward kernel (the traffic record goes stale when
-# either file changes).
+# Device code of the timed forward kernel: the traffic record goes stale when
+# the code in either file changes (comments and blank lines do not count).
 FWD_KERNEL_SOURCES = ("attn_fwd_kernel.cuh", "sm100.cuh")
+
+
+def strip_comments(src: str) -> str:
+    """C++ source without // and /* */ comments, trailing blanks and blank
+    lines; string and character literals are kept as they are."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            end = src.find("*/", i + 2)
+            i = n if end < 0 else end + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [line.rstrip() for line in "".join(out).split("\n")]
+    return "\n".join(line for line in lines if line)
 
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_softmax_attention_04_b200", "csrc")
     for f in FWD_KERNEL_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,9 +17,9 @@
 // Roles (384 threads, 12 warps = 3 warpgroups, one warp of each per SMSP):
 //   warps 0-3  softmax for Q_0; warps 4-7 softmax for Q_1. Thread r of a
 //              warpgroup owns query row r (= TMEM lane r): it reads its S row,
-//              masks boundary tiles, updates (m, l), writes P (bf16) back into
-//              TMEM over its S columns, rescales its O row when m grew, and runs
-//              the epilogue (O / l -> bf16 -> smem -> TMA store; LSE store).
+//              masks boundary tiles, updates (m, l), writes P (bf16) into TMEM,
+//              rescales its O row when m grew, and runs the epilogue
+//              (O / l -> bf16 -> smem -> TMA store; LSE store).
 //   warp 8     MMA issuer (one elected lane) and TMEM owner.
 //   warp 9     TMA producer (one elected lane): Q_0, Q_1 once, then K_j, V_j
 //              alternately into a ring of NSLOT shared-memory slots.
@@ -27,14 +27,21 @@
 // Registers: launched at 168 per thread; the softmax warpgroups raise theirs
 // to 232 (a 128-float S row plus its P stay in registers, no spills) and the
 // third warpgroup drops to 40: 2*128*232 + 128*40 = 384*168.
-// TMEM columns: S_0/P_0 [0,128), S_1/P_1 [128,256), O_0 [256, 256+D),
-// O_1 [256+D, 256+2D).
-// MMA issue order per key tile j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j). The
-// two softmax warpgroups thus alternate with the tensor core: while one works
-// on its S, the tensor core runs the other tile's PV and S. tcgen05 MMAs from
-// one thread complete in issue order, so (a) S_s(j) overwrites P_s(j-1) only
-// after PV_s(j-1) has read it, and (b) when S_s(j) is complete, PV_s(j-1) is
-// too, so the softmax may rescale O_s right away.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256, 256+D),
+// O_1 [256+D, 256+2D); P_s over S_s at D = 128, in its own columns at D = 64
+// (P_0 [384,448), P_1 [448,512)).
+// MMA issue order per key tile j, D = 128: PV_0(j-1), S_0(j), PV_1(j-1),
+// S_1(j). tcgen05 MMAs from one thread complete in issue order, so (a) S_s(j)
+// overwrites P_s(j-1) only after PV_s(j-1) has read it, and (b) when S_s(j)
+// is complete, PV_s(j-1) is too, so the softmax may rescale O_s right away.
+// D = 64: S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), S_s(j) waiting only until the
+// softmax has read S_s(j-1) into registers; the softmax waits for PV_s(j-1)
+// before it overwrites P_s or rescales O_s.
+// The exponentials run on the MUFU, and on unmasked tiles a fixed share of
+// them on the FMA pipe as a polynomial (see ex2_poly_x2); the share and the
+// form of the row max differ per head size (FwdCfg).
+// Two instantiations: BLOCKMASK = false for the causal and window masks (the
+// closed-form bounds), true for the block-local mask (Mask intervals).
 //
 // Every wait is bounded (about one second). On expiry the kernel sets bit 1
 // of the device status word, tells the other roles to stop, waits (bounded)
