@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
                 break;
             const int slot = s0 + (issued / 2) * DEC_TK;
             const CUtensorMap *map = (issued & 1) ? &tmV : &tmK;
+#ifdef ATTN_FAULT_DEC_DROP_FIRST_K
+            // Test hook (never defined in the library build): the first K
+            // tile is never loaded, so every wait on it must expire and the
+            // kernel must stop cleanly.
+            if (issued == 0) continue;
+#endif
             mbar_arrive_expect_tx_if(leader, full(st), C::TILE_BYTES);
 #pragma unroll
             for (int bx = 0; bx < C::BOXES; ++bx)
@@ -291,7 +297,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2)
                     if (lane == 0) red[(sb * 4 + sw) * 8 + g] = mx;
                 }
             }
-            ok = named_bar_and(1, 4 * 32, okw);
+            // (ok carries a wait that gave up later in the previous tile)
+            ok = named_bar_and(1, 4 * 32, okw && ok);
             if (!ok) break;
             const int slot0 = s0 + i * DEC_TK;
             const bool valid = slot0 + r < s1;

@@ -1,11 +1,12 @@
 """Failure detection without faulting the GPU.
 
-Every wait in the kernel is bounded (about one second). A build with the
-test-only ATTN_FAULT_DROP_FIRST_V hook never loads the first V tile, so the
-MMA warp's wait for it must expire: the kernel then sets the device status
-word, stops all roles, waits (bounded) for what it issued, frees TMEM and
-returns. The host must read ATTN_ERR_TIMEOUT, the status must clear, and the
-CUDA context must stay usable for a correct computation afterwards.
+Every wait in the kernels is bounded (about one second). Builds with a
+test-only hook never load one tile (forward: the first V tile; backward: the
+first Q/dO stage; decode: the first K tile), so a wait for it must expire:
+the kernel then sets the device status word, stops all roles, waits
+(bounded) for what it issued, frees TMEM and returns. The host must read
+ATTN_ERR_TIMEOUT, the status must clear, and the CUDA context must stay
+usable for a correct computation afterwards.
 """
 import time
 
@@ -83,3 +84,40 @@ def test_backward_expired_wait_reports_timeout_and_context_survives(tmp_path, or
     assert pkg.sync_status() == pkg.ATTN_OK
     refs = oracle_mod.attn_bwd(q, k, v, do, 0.125, True, -1)
     assert_grads_close([g.float().cpu().numpy() for g in grads], refs, "after backward timeout")
+
+
+def test_decode_expired_wait_reports_timeout_and_context_survives(tmp_path, oracle_mod):
+    """The decode kernel's first K tile is never loaded (test-only
+    ATTN_FAULT_DEC_DROP_FIRST_K hook): the MMA warp's and the softmax warps'
+    waits on it must expire, the call must report ATTN_ERR_TIMEOUT, and the
+    context must stay usable."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import exact_softmax_attention_04_b200 as pkg
+    from exact_softmax_attention_04_b200 import build_lib
+    build_lib.build()
+    fault_lib = pkg.load_library(build_lib.build_variant(tmp_path / "libattn_fault_dec.so",
+                                                         ["ATTN_FAULT_DEC_DROP_FIRST_K"]))
+    # four CTAs (four splits of one 128-slot tile each), four query heads per K/V head
+    B, H, Hkv, W, d = 1, 4, 1, 512, 128
+    q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=52, q_std=1.0)
+    qd, kd, vd = q.cuda(), kc.cuda(), vc.cuda()
+    pos = torch.tensor([W - 1], dtype=torch.int32, device="cuda")
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    ws = torch.empty(pkg.decode_workspace_bytes(B, H, Hkv, W, d), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    sc = 1.0 / np.sqrt(d)
+    t0 = time.time()
+    rc = fault_lib.attn_decode(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), pos.data_ptr(), o.data_ptr(),
+                               lse.data_ptr(), ws.data_ptr(), ws.numel(), B, H, Hkv, W, d, sc, stream)
+    assert rc == pkg.ATTN_OK
+    st = fault_lib.attn_sync_status(stream)
+    assert st == pkg.ATTN_ERR_TIMEOUT, pkg.strerror(st)
+    assert time.time() - t0 < 30.0
+    assert fault_lib.attn_sync_status(stream) == pkg.ATTN_OK
+    o2, lse2 = pkg.attn_decode(qd, kd, vd, pos, sc)
+    assert pkg.sync_status() == pkg.ATTN_OK
+    o_ref, lse_ref = oracle_mod.attn_decode(q, kc, vc, [W - 1], sc)
+    assert_close(o2.float().cpu().numpy().reshape(-1, d), lse2.cpu().numpy().reshape(-1),
+                 o_ref.reshape(-1, d), lse_ref.reshape(-1), "after decode timeout")
