@@ -100,9 +100,16 @@ Staging g_staging[kMaxDevices];
 
 // Side streams of attn_fwd_host, one per copy direction, so that one chunk
 // of heads is copied in while another is computed and a third copied out.
-constexpr int kHostChunks = 8;
+#ifndef ATTN_HOST_CHUNKS
+#define ATTN_HOST_CHUNKS 8
+#endif
+#ifndef ATTN_HOST_H2D_STREAMS
+#define ATTN_HOST_H2D_STREAMS 1
+#endif
+constexpr int kHostChunks = ATTN_HOST_CHUNKS;
+constexpr int kH2D = ATTN_HOST_H2D_STREAMS;  // copy-in streams, used by chunks in turn
 struct HostPipe {
-    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaStream_t h2d[kH2D] = {}, d2h = nullptr;
     cudaEvent_t entry = nullptr, done = nullptr;
     cudaEvent_t in[kHostChunks] = {}, ran[kHostChunks] = {};
     bool ready = false;
@@ -115,14 +122,17 @@ int host_pipe(int dev, HostPipe **out)
 {
     HostPipe &hp = g_pipe[dev];
     if (!hp.ready) {
-        bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&hp.entry, cudaEventDisableTiming) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
-        for (int c = 0; ok && c < kHostChunks; ++c)
-            ok = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
-                 cudaEventCreateWithFlags(&hp.ran[c], cudaEventDisableTiming) == cudaSuccess;
-        if (!ok) return ATTN_ERR_CUDA;  // what was created is kept and reused next time
+        // each handle is created once; after a failure, what exists is kept
+        auto stream = [](cudaStream_t &h) {
+            return h || cudaStreamCreateWithFlags(&h, cudaStreamNonBlocking) == cudaSuccess;
+        };
+        auto event = [](cudaEvent_t &e) {
+            return e || cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+        };
+        bool ok = stream(hp.d2h) && event(hp.entry) && event(hp.done);
+        for (int i = 0; ok && i < kH2D; ++i) ok = stream(hp.h2d[i]);
+        for (int c = 0; ok && c < kHostChunks; ++c) ok = event(hp.in[c]) && event(hp.ran[c]);
+        if (!ok) return ATTN_ERR_CUDA;
         hp.ready = true;
     }
     *out = &hp;
@@ -331,17 +341,19 @@ extern "C" int attn_fwd_host(const void *q, const void *k, const void *v, void *
     // Side-stream work starts after everything already on `stream` (the
     // staging buffers may still be in use by an earlier call), and `stream`
     // continues only once the last copy-out is done.
-    if (cudaEventRecord(hp->entry, st) != cudaSuccess || cudaStreamWaitEvent(hp->h2d, hp->entry, 0) != cudaSuccess)
-        return ATTN_ERR_CUDA;
+    if (cudaEventRecord(hp->entry, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    for (int i = 0; i < kH2D; ++i)
+        if (cudaStreamWaitEvent(hp->h2d[i], hp->entry, 0) != cudaSuccess) return ATTN_ERR_CUDA;
     for (int c = 0; c < chunks; ++c) {
         const int64_t h0 = c * per;
         const int hc = static_cast<int>(bh - h0 < per ? bh - h0 : per);
         const size_t off = static_cast<size_t>(h0) * head_bytes, bytes = static_cast<size_t>(hc) * head_bytes;
         const size_t loff = static_cast<size_t>(h0) * n, lbytes = static_cast<size_t>(hc) * n * 4;
-        if (cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-            cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-            cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
-            cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp->in[c], 0) != cudaSuccess)
+        cudaStream_t in_st = hp->h2d[c % kH2D];
+        if (cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, in_st) != cudaSuccess ||
+            cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, in_st) != cudaSuccess ||
+            cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, in_st) != cudaSuccess ||
+            cudaEventRecord(hp->in[c], in_st) != cudaSuccess || cudaStreamWaitEvent(st, hp->in[c], 0) != cudaSuccess)
             return ATTN_ERR_CUDA;
         rc = attn_fwd(dq + off, dk + off, dv + off, dout + off, dl + loff, 1, hc, n, d, scale, causal, window,
                       stream);
