@@ -120,9 +120,9 @@ ATTN_API int attn_fwd_gqa(const void *q, const void *k, const void *v, void *o, 
  * blocks of `block` consecutive tokens, query i attends to the keys of its
  * own block and of the previous one, floor(j/block) in {floor(i/block) - 1,
  * floor(i/block)}, and only to j <= i when causal = 1 (the block-sparse
- * pattern of "Sparse & sub-quadratic attention", section "Escape 1":
- * attend within your block and the previous one). A block of n tokens or
- * more is one block: the same keys as attn_fwd without a window.
+ * pattern of "Sparse & sub-quadratic attention", section "Escape 1": a
+ * token sees the keys of its own block and of the block before). A block of
+ * n tokens or more is one block: the same keys as attn_fwd without a window.
  *
  *   block  : >= 1 (else ATTN_ERR_INVALID)
  *   Hkv    : key/value heads, as attn_fwd_gqa (Hkv = H for multi-head)

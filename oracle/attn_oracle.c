@@ -27,7 +27,7 @@
  *   block-local (block b > 0, no window) : floor(j/b) is floor(i/b) or
  *            floor(i/b) - 1, and j <= i as well when causal (the block-sparse
  *            pattern of "Sparse & sub-quadratic attention", section "Escape 1":
- *            attend within your block and the previous one)
+ *            a token sees the keys of its own block and of the block before)
  * Then, all in fp64 over the bf16-decoded inputs,
  *   s_ij  = scale * sum_c q_ic k_jc          for j in A(i)
  *   M_i   = max_{j in A(i)} s_ij

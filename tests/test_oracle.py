@@ -227,10 +227,8 @@ def test_associativity_identity_escape2(oracle_mod):
     g = _golden("associativity_escape2.txt")
     N, d = int(g["N"]), int(g["d"])
     assert N * N == int(g["nxn_floats"]) and d * d == int(g["dxd_floats"])
-    rng = np.random.default_rng(0)
-    Q = rng.standard_normal((N, d))
-    K = rng.standard_normal((N, d))
-    V = rng.standard_normal((N, d))
+    # three N x d standard-normal matrices (the worked example's sizes)
+    Q, K, V = np.random.default_rng(0).standard_normal((3, N, d))
     A = oracle_mod.matmul(oracle_mod.matmul(Q, K, tb=True), V)
     Bm = oracle_mod.matmul(Q, oracle_mod.matmul(K, V, ta=True))
     assert str(bool(np.allclose(A, Bm))) == g["allclose"]
