@@ -1,7 +1,6 @@
 """The C ABI boundary, checked without a GPU: the library builds and loads,
 exports every function include/attn.h declares, and rejects bad arguments
 before touching the device."""
-import ctypes
 import os
 import re
 import subprocess
