@@ -1,7 +1,7 @@
 /*
  * attn.h - C ABI of the B200 (sm_100a) exact softmax attention library
- * (libattn_b200.so): forward pass, grouped-query forward, backward pass,
- * decode against rolling key/value caches.
+ * (libattn_b200.so): forward pass (device or host buffers), grouped-query and
+ * block-local forms, backward pass, decode against rolling key/value caches.
  *
  * The operation (all entry points that compute):
  *
@@ -41,13 +41,16 @@
  *
  * Ownership: the caller owns every buffer passed in and keeps it alive until
  * the work enqueued on `stream` has finished. The library owns only: one
- * lazily allocated device status word per device, and, for attn_fwd_host, a
+ * lazily allocated device status word per device; for attn_fwd_host, a
  * per-device set of device staging buffers (grown on demand, released by
- * attn_host_staging_release). No entry point prints, exits, aborts or traps.
+ * attn_host_staging_release) and two side streams with their events (created
+ * once per device); for attn_fwd_host_noalloc, one static device array per
+ * device. No entry point prints, exits, aborts or traps.
  *
  * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  * stream). Work is enqueued on it on the calling thread's current device; the
- * device pointers must belong to that device.
+ * device pointers must belong to that device. attn_fwd_host also runs copies
+ * on its side streams, ordered with `stream` by events (see there).
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -221,7 +224,7 @@ ATTN_API int attn_fwd_host_noalloc(const void *q, const void *k, const void *v, 
  *                      its contents on entry do not matter, and it must not
  *                      be used by other work until this call's work is done
  *   B, H, n, d, scale, causal, window, stream : as attn_fwd (K and V have H
- *                      heads: the grouped-query form has no backward here)
+ *                      heads; attn_bwd_gqa below is the grouped-query form)
  *
  * Arithmetic: bf16 tensor-core products with fp32 accumulation; P and dS
  * are rounded to bf16 before their products; all sums are fp32 and each
