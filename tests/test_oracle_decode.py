@@ -76,3 +76,18 @@ def test_decode_oracle_rejects_bad_arguments(oracle_mod):
     q3, kc3, vc3 = synth.make_decode(1, 4, 3, 8, 16, seed=8)
     with pytest.raises(ValueError):
         oracle_mod.attn_decode(q3, kc3, vc3, [0], 0.25)  # 3 does not divide 4
+
+
+def test_unused_slots_never_read(oracle_mod):
+    """Slots no position has reached yet (slot >= pos + 1 while pos < W - 1)
+    may hold anything: NaN there leaves the result bit for bit unchanged."""
+    B, H, Hkv, W, d = 3, 4, 2, 40, 16
+    q, kc, vc = synth.make_decode(B, H, Hkv, W, d, seed=21, q_std=1.5)
+    pos = [0, 17, 38]
+    o_ref, l_ref = oracle_mod.attn_decode(q, kc, vc, pos, 0.3)
+    kn, vn = kc.clone(), vc.clone()
+    for b, t in enumerate(pos):
+        kn[b, :, t + 1:] = float("nan")
+        vn[b, :, t + 1:] = float("nan")
+    o, l = oracle_mod.attn_decode(q, kn, vn, pos, 0.3)
+    assert np.array_equal(o, o_ref) and np.array_equal(l, l_ref)
