@@ -3,14 +3,20 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                 [--workload NAME]
 
-One step = one attention forward (the whole hot path: one kernel launch) over
-the workload B=8, H=8, n=8192, d=64, no mask, bf16 Q/K/V ~ N(0,1) from seed 0
-(the 8x8x8192 worked example of "Quadratic cost and efficient attention",
-d_model 512 over 8 heads). FLOPs counted: 4*d per attended (query, key) pair.
-Inputs (201 MB) and outputs exceed the 126 MB L2, so no explicit flush is
-done between steps. Under torchrun every rank runs its own replica (the work
-shards by (batch, head) with no exchange), so scaling is weak and the value is
-the sum of all ranks' FLOPs over the slowest rank's time.
+One step = one attention forward (the whole hot path: one kernel launch).
+Default workload: B=1, H=8, n=131072, d=128, full causal mask, bf16 Q/K/V ~
+N(0,1) from seed 0 -- the long-context stress case and the largest of the
+target configurations that fits one GPU (the cost of long contexts is the
+subject of "Quadratic cost and efficient attention", section "What long
+context really costs"). Other workloads by name with --workload, e.g.
+B8-H8-n8192-d64-none (the 8x8x8192 worked example of the same page, d_model
+512 over 8 heads) or B1-H32-n32768-d128-window4096 (Mistral's w = 4096).
+FLOPs counted: 4*d per attended (query, key) pair. Inputs and outputs of the
+default workload (0.8 GB in, 0.27 GB out) exceed the 126 MB L2, so no
+explicit flush is done between steps. Under torchrun every rank runs its own
+replica (the work shards by (batch, head) with no exchange), so scaling is
+weak and the value is the sum of all ranks' FLOPs over the slowest rank's
+time.
 
 --impl reference times the fp64 CPU oracle on a bounded row sample of the
 same workload (rank 0 only): the deliberately slow reference arm.
@@ -35,6 +41,8 @@ METRIC = "attention fwd TFLOP/s (unmasked FLOPs) and % of B200 dense BF16 peak"
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_NAME = "attn_fwd_kernel"
+# the largest target configuration that fits one GPU
+DEFAULT_WORKLOAD = "B1-H8-n131072-d128-causal"
 
 
 def _env_int(name, default):
@@ -209,6 +217,29 @@ def replica_throughput(units_per_rank: float, steps: int, max_ms: float, world: 
     return world * units_per_rank * steps / (max_ms / 1e3)
 
 
+def head_shard(bh: int, world: int, rank: int):
+    """Contiguous range [start, stop) of the flattened (batch, head) pairs that
+    `rank` of `world` owns when one problem is split across ranks: every
+    (batch, head) pair is an independent attention problem, so the ranks
+    need no exchange and their outputs are disjoint slices. Earlier ranks
+    take one extra pair when bh does not divide evenly."""
+    base, extra = divmod(bh, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def workload_config(wl, world: int) -> dict:
+    """The `config` object of a JSON line, identical for both arms: the
+    workload, its size per replica and how L2 is handled between steps."""
+    elems = wl.B * wl.H * wl.n * wl.d
+    in_bytes = 2 * elems + 2 * 2 * wl.B * wl.kv_heads * wl.n * wl.d
+    out_bytes = 2 * elems + 4 * wl.B * wl.H * wl.n
+    return {**wl.describe(), "global_batch": wl.B * world, "seq_len": wl.n,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"no flush: inputs {in_bytes / 1e6:.0f} MB + outputs {out_bytes / 1e6:.0f} MB per step "
+                  + ("exceed" if in_bytes > 126e6 else "do NOT exceed") + " the 126 MB L2"}
+
+
 def cpu_baseline_leg(wl, o_gpu=None, lse_gpu=None, target_s: float = 15.0):
     """Oracle timed on this host's cores over a bounded row sample of the
     workload; also compares those rows with the GPU outputs if given."""
@@ -284,7 +315,8 @@ def run_reference(args, wl, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**wl.describe(), "l2": "n/a (CPU)"},
+        "config": workload_config(wl, world),
+        "note": "the fp64 oracle on the host cores; no GPU and no L2 involved",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -405,7 +437,6 @@ def run_ours(args, wl, world, rank, local):
 
     if rank != 0:
         return 0
-    in_bytes = q.numel() * 2 + 2 * k.numel() * 2
     sustained = None
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -420,11 +451,7 @@ def run_ours(args, wl, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {**wl.describe(), "global_batch": wl.B * world, "seq_len": wl.n,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"no flush: inputs {in_bytes / 1e6:.0f} MB + outputs "
-                         f"{(o.numel() * 2 + lse.numel() * 4) / 1e6:.0f} MB per step "
-                         + ("exceed" if in_bytes > 126e6 else "do NOT exceed") + " the 126 MB L2"},
+        "config": workload_config(wl, world),
         "pct_of_peak": 100.0 * value / world / bf16_peak,
         "roofline": roofline,
         "e2e": e2e,
@@ -697,7 +724,7 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="B8-H8-n8192-d64-none")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="oracle work budget of the --impl reference arm (warm-up and timed steps)")

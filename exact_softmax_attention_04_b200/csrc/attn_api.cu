@@ -495,5 +495,8 @@ extern "C" int attn_fwd_host_noalloc(const void *q, const void *k, const void *v
     if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
     int h = 0;
     if (cudaMemcpy(&h, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
-    return h != 0 ? ATTN_ERR_TIMEOUT : ATTN_OK;
+    // The same reading of the status bits as attn_sync_status: bit 1 means a
+    // bounded wait expired, any other bit that a kernel refused to run.
+    if (h == 0) return ATTN_OK;
+    return (h & attn_sm100::STATUS_WAIT_TIMEOUT) ? ATTN_ERR_TIMEOUT : ATTN_ERR_CUDA;
 }

@@ -3,8 +3,8 @@
 // Each sequence b has one query token at position t = pos[b]; its keys and
 // values sit in a W-slot rolling cache, position p in slot p mod W, so the
 // cache holds positions max(0, t - W + 1) .. t (the rolling buffer of the
-// worked example on "Sparse & sub-quadratic attention": a 4,096-position
-// cache serving n = 32,768). Softmax is invariant to the order of its terms,
+// worked example on "Beyond attention", section "For engineers -- Show the
+// maths": a 4,096-position cache serving n = 32,768). Softmax is invariant to the order of its terms,
 // so the query attends to slots [0, L) with L = min(t + 1, W), in slot order.
 // Query head h reads key/value head h / G, G = H / Hkv (grouped-query
 // attention, "week17 efficiency attention", MQA / GQA section).

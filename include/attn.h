@@ -182,8 +182,11 @@ ATTN_API int attn_host_staging_release(void);
  *   Limit: 4 * B*H*n*d*2 + B*H*n*4 bytes (each part rounded up to 256) plus
  *          256 must fit in ATTN_NOALLOC_SCRATCH_BYTES; larger problems return
  *          ATTN_ERR_TOO_LARGE before any device work.
- *   Synchronous: returns once o and lse are written (it synchronizes
- *          `stream`), with ATTN_ERR_TIMEOUT if the kernel gave up a wait.
+ *   Synchronous: the call waits for its own copies and kernel to finish
+ *          (it synchronizes `stream`) and returns once o and lse hold the
+ *          result. ATTN_ERR_TIMEOUT if the kernel gave up a bounded wait,
+ *          ATTN_ERR_CUDA if a kernel refused to run (the status word read
+ *          as attn_sync_status reads it).
  *   Set-up: the first call on a device looks up the array's device address
  *          (cudaGetSymbolAddress) with that device current; make that first
  *          call before any stream capture.
@@ -284,8 +287,8 @@ ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
  * position p is stored in slot p mod W, so after the current token's own
  * key and value have been written the cache holds positions
  * max(0, pos[b] - W + 1) .. pos[b] (the rolling buffer of the worked example
- * on "Sparse & sub-quadratic attention": a 4,096-position cache serving
- * n = 32,768). The query attends to exactly those positions:
+ * on "Beyond attention", section "For engineers -- Show the maths": a
+ * 4,096-position cache serving n = 32,768). The query attends to exactly those positions:
  *
  *   O[b,h]   = softmax(scale * q[b,h] . k) v   over the cached positions,
  *   LSE[b,h] = ln sum exp(scale * q[b,h] . k)  (natural-log units),

@@ -524,9 +524,9 @@ int oracle_attn_bwd_rows_f64(const void *q, const void *k, const void *v, const 
  * Decode against a rolling key/value cache.
  *
  * One query token per sequence attends to the keys a sliding window keeps.
- * The cache is the rolling buffer of "Sparse & sub-quadratic attention"
- * (worked example of the maths panel: a 4,096-position cache serving
- * n = 32,768, after Mistral): W slots per key/value head, position p stored
+ * The cache is the rolling buffer of "Beyond attention" (section "For
+ * engineers -- Show the maths", worked example: a 4,096-position cache
+ * serving n = 32,768, after Mistral): W slots per key/value head, position p stored
  * at slot p mod W, so after writing position t the cache holds positions
  * max(0, t - W + 1) .. t. For sequence b with query position t = pos[b] and
  * query head h (key/value head h / (H / Hkv), as for grouped-query
