@@ -63,6 +63,9 @@ def _load():
         lib.oracle_attn_bwd_rows_gqa_f64.restype = ip
         lib.oracle_attn_decode_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp]
         lib.oracle_attn_decode_f64.restype = ip
+        lib.oracle_attn_decode_multi_f64.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, dbl,
+                                                     vp, vp]
+        lib.oracle_attn_decode_multi_f64.restype = ip
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ip
         _lib = lib
@@ -245,6 +248,33 @@ def attn_decode(q, k_cache, v_cache, pos, scale: float) -> Tuple[np.ndarray, np.
                                     B, H, Hkv, W, d, float(scale), o.ctypes.data, lse.ctypes.data)
     if rc != 0:
         raise ValueError(f"oracle_attn_decode_f64 rejected its arguments (rc={rc})")
+    return o, lse
+
+
+def attn_decode_multi(q, k_cache, v_cache, pos, scale: float, window: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Decode of T new tokens per sequence against rolling caches: q bf16
+    [B, H, T, d] (token u at position pos[b] - T + 1 + u), k_cache / v_cache
+    bf16 [B, Hkv, W, d] (position p at slot p mod W), pos [B] (>= T - 1, the
+    last new token's position), causal window `window` (window + T <= W).
+    Returns O [B, H, T, d] and LSE [B, H, T] in fp64."""
+    lib = _load()
+    if len(q.shape) != 4 or len(k_cache.shape) != 4 or k_cache.shape != v_cache.shape:
+        raise ValueError("q must be [B, H, T, d] and the caches [B, Hkv, W, d]")
+    B, H, T, d = q.shape
+    Bk, Hkv, W, dk = k_cache.shape
+    if Bk != B or dk != d:
+        raise ValueError("cache shape does not match q")
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    p = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    if p.size != B:
+        raise ValueError("pos must have B entries")
+    o = np.empty((B, H, T, d), dtype=np.float64)
+    lse = np.empty((B, H, T), dtype=np.float64)
+    rc = lib.oracle_attn_decode_multi_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, p.ctypes.data,
+                                          B, H, Hkv, T, W, d, int(window), float(scale), o.ctypes.data,
+                                          lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_decode_multi_f64 rejected its arguments (rc={rc})")
     return o, lse
 
 

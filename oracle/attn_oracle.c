@@ -597,3 +597,82 @@ int oracle_attn_decode_f64(const uint16_t *q, const uint16_t *k, const uint16_t 
     }
     return bad ? 2 : 0;
 }
+
+/* ========================================================================
+ * Decode of a few new tokens per sequence against a rolling cache.
+ *
+ * The same rolling buffer as above (position p in slot p mod W), now with T
+ * new query tokens per sequence, at positions t_u = pos[b] - T + 1 + u for
+ * u = 0 .. T-1 (pos[b] is the last of them; all T have been written to the
+ * cache before the step). Token u attends causally within the new tokens and
+ * to the sliding window of w earlier positions (the causal window-w mask of
+ * "week17 efficiency attention", local attention section):
+ *   A(u) = { p : max(0, t_u - w) <= p <= t_u },
+ * so the T outputs are rows t_0 .. t_{T-1} of the causal window-w forward
+ * pass over the sequence that filled the cache. Every p in A(u) is still in
+ * the cache only if w + T <= W (the oldest needed position, t_0 - w, is then
+ * at least pos - W + 1); the oracle rejects other arguments. T = 1 and
+ * w = W - 1 is the single-token decode above.
+ *   s_p  = scale * q_u . k(slot p mod W),  M = max_{p in A(u)} s_p,
+ *   O    = sum_{p in A(u)} exp(s_p - M) v(slot p mod W) / sum exp(s_p - M),
+ *   LSE  = M + ln sum_{p in A(u)} exp(s_p - M).
+ *   q : bf16 [B, H, T, d];  k, v : bf16 [B, Hkv, W, d];  pos : int64 [B], >= T - 1
+ *   o : fp64 [B, H, T, d];  lse : fp64 [B, H, T]
+ * ======================================================================== */
+int oracle_attn_decode_multi_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int64_t *pos,
+                                 int64_t B, int64_t H, int64_t Hkv, int64_t T, int64_t W, int64_t d,
+                                 int64_t window, double scale, double *o, double *lse)
+{
+    if (!q || !k || !v || !pos || !o || !lse || B <= 0 || H <= 0 || Hkv <= 0 || T <= 0 || W <= 0 || d <= 0)
+        return 1;
+    if (H % Hkv != 0 || window < 0 || window + T > W)
+        return 1;
+    for (int64_t b = 0; b < B; ++b)
+        if (pos[b] < T - 1)
+            return 1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(window + 1));
+        if (!s) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t row = 0; row < B * H * T; ++row) {
+                const int64_t bh = row / T, u = row % T;
+                const int64_t b = bh / H, h = bh % H;
+                const int64_t kvh = b * Hkv + h / (H / Hkv);
+                const int64_t t = pos[b] - T + 1 + u;           /* this token's position */
+                const int64_t first = (t - window > 0) ? t - window : 0;
+                const int64_t count = t - first + 1;
+                const uint16_t *qr = q + row * d;
+                double M = -INFINITY;
+                for (int64_t i = 0; i < count; ++i) {
+                    const uint16_t *kr = k + (kvh * W + (first + i) % W) * d;
+                    double acc = 0.0;
+                    for (int64_t c = 0; c < d; ++c)
+                        acc += bf16_to_f64(qr[c]) * bf16_to_f64(kr[c]);
+                    s[i] = scale * acc;
+                    if (s[i] > M)
+                        M = s[i];
+                }
+                double Z = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    o[row * d + c] = 0.0;
+                for (int64_t i = 0; i < count; ++i) {
+                    const uint16_t *vr = v + (kvh * W + (first + i) % W) * d;
+                    const double w = exp(s[i] - M);
+                    Z += w;
+                    for (int64_t c = 0; c < d; ++c)
+                        o[row * d + c] += w * bf16_to_f64(vr[c]);
+                }
+                for (int64_t c = 0; c < d; ++c)
+                    o[row * d + c] /= Z;
+                lse[row] = M + log(Z);
+            }
+        }
+        free(s);
+    }
+    return bad ? 2 : 0;
+}
