@@ -580,28 +580,37 @@ DECODE_METRIC = "decode GB/s (cached K and V read once, plus q, O, LSE)"
 
 
 def run_decode(args, wl, world, rank, local):
-    """One decode step against rolling caches (attn_decode: split kernel and
+    """One decode step against rolling caches (attn_decode, or
+    attn_decode_multi for several new tokens per sequence: split kernel and
     merge) per step, timed like the forward; the roofline is HBM bandwidth on
-    the algorithmic bytes: the cached keys and values each query group
-    attends to, read once, plus q, O and LSE."""
+    the algorithmic bytes: the cached keys and values, read once, plus q, O
+    and LSE."""
     import numpy as np
     import exact_softmax_attention_04_b200 as attn
     from exact_softmax_attention_04_b200 import synth
 
     dev = torch.device("cuda", local)
-    q, kc, vc = synth.make_decode(wl.B, wl.H, wl.Hkv, wl.W, wl.d, seed=wl.seed, q_std=wl.q_std)
+    multi = wl.T > 1 or wl.w != wl.W - 1
+    if multi:
+        q, kc, vc = synth.make_decode_multi(wl.B, wl.H, wl.Hkv, wl.T, wl.W, wl.d, seed=wl.seed, q_std=wl.q_std)
+    else:
+        q, kc, vc = synth.make_decode(wl.B, wl.H, wl.Hkv, wl.W, wl.d, seed=wl.seed, q_std=wl.q_std)
     qd, kd, vd = q.to(dev), kc.to(dev), vc.to(dev)
     pos = torch.full((wl.B,), wl.pos, dtype=torch.int32, device=dev)
     o = torch.empty_like(qd)
-    lse = torch.empty((wl.B, wl.H), dtype=torch.float32, device=dev)
-    ws = torch.empty(attn.decode_workspace_bytes(wl.B, wl.H, wl.Hkv, wl.W, wl.d), dtype=torch.uint8, device=dev)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_multi_workspace_bytes(wl.B, wl.H, wl.Hkv, wl.T, wl.W, wl.w, wl.d),
+                     dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     nbytes = 2 * wl.B * wl.Hkv * wl.keys * wl.d * 2 + 2 * q.numel() * 2 + lse.numel() * 4
-    flops = 4 * wl.d * wl.keys * wl.B * wl.H
+    flops = 4 * wl.d * wl.attended * wl.B * wl.H
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
-        attn.attn_decode(qd, kd, vd, pos, wl.scale, out=o, lse=lse, workspace=ws, stream=stream)
+        if multi:
+            attn.attn_decode_multi(qd, kd, vd, pos, wl.w, wl.scale, out=o, lse=lse, workspace=ws, stream=stream)
+        else:
+            attn.attn_decode(qd, kd, vd, pos, wl.scale, out=o, lse=lse, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -649,7 +658,7 @@ def run_decode(args, wl, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": gbs / hbm_peak, "traffic": None, "peak_source": f"{peak_src} HBM copy",
                      "algorithmic_bytes_per_launch": nbytes,
-                     "note": "achieved over the attn_decode call (split kernel and merge kernel)"},
+                     "note": "achieved over the decode call (split kernel and merge kernel)"},
         "e2e": {"value": None, "unit": "GB/s", "note": "decode has no host-buffer entry point"},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(wall0, wall1),
@@ -660,7 +669,11 @@ def run_decode(args, wl, world, rank, local):
         g = torch.Generator().manual_seed(2)
         nseq = max(1, min(wl.B, 4))
         t0 = time.perf_counter()
-        o_ref, lse_ref = oracle.attn_decode(q[:nseq], kc[:nseq], vc[:nseq], [wl.pos] * nseq, wl.scale)
+        if multi:
+            o_ref, lse_ref = oracle.attn_decode_multi(q[:nseq], kc[:nseq], vc[:nseq], [wl.pos] * nseq, wl.scale,
+                                                      wl.w)
+        else:
+            o_ref, lse_ref = oracle.attn_decode(q[:nseq], kc[:nseq], vc[:nseq], [wl.pos] * nseq, wl.scale)
         dt = time.perf_counter() - t0
         og = o[:nseq].float().cpu().numpy()
         line["cpu_baseline"] = {
@@ -732,8 +745,10 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="time every target workload (kernel only, median of --steps, L2 flushed)")
     ap.add_argument("--decode", action="store_true",
-                    help="time one decode step against rolling caches (attn_decode); --workload "
-                         "defaults to decode-B64-H32-Hkv8-W4096-d128-pos32767")
+                    help="time one decode step against rolling caches; --workload defaults to "
+                         "decode-B64-H32-Hkv8-W4096-d128-pos32767 (one new token, attn_decode); "
+                         "decode-B64-H32-Hkv8-T4-W4096-w4092-d128-pos32767 takes four new tokens per "
+                         "sequence (attn_decode_multi)")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (attn_bwd) of --workload instead of the forward")
     ap.add_argument("--profile", action="store_true",

@@ -30,7 +30,8 @@ ATTN_ERR_TOO_LARGE = 5
 EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_release",
            "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
            "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes", "attn_decode",
-           "attn_decode_workspace_bytes", "attn_fwd_blocklocal", "attn_bwd_blocklocal")
+           "attn_decode_workspace_bytes", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
+           "attn_fwd_blocklocal", "attn_bwd_blocklocal")
 
 
 class AttnError(RuntimeError):
@@ -85,6 +86,10 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_decode.restype = i
     lib.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.attn_decode_workspace_bytes.restype = i64
+    lib.attn_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, i, i, f, vp]
+    lib.attn_decode_multi.restype = i
+    lib.attn_decode_multi_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    lib.attn_decode_multi_workspace_bytes.restype = i64
     return lib
 
 
@@ -280,6 +285,53 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
                                _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_decode")
+    return out, lse
+
+
+def decode_multi_workspace_bytes(B: int, H: int, Hkv: int, T: int, W: int, window: int, d: int) -> int:
+    r = int(lib().attn_decode_multi_workspace_bytes(int(B), int(H), int(Hkv), int(T), int(W), int(window),
+                                                    int(d)))
+    if r < 0:
+        raise ValueError("unsupported or invalid shape for attn_decode_multi")
+    return r
+
+
+def attn_decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, pos: torch.Tensor,
+                      window: int, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """A decode step of T new tokens per sequence: q bf16 [B, H, T, d] (token
+    u at position pos[b] - T + 1 + u), rolling caches k_cache / v_cache bf16
+    [B, Hkv, W, d], pos int32 [B] on the device (each sequence's last new
+    token), causal window `window` (window + T <= W). Returns (o bf16
+    [B, H, T, d], lse fp32 [B, H, T]); see include/attn.h."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if q.dim() != 4 or k_cache.dim() != 4 or k_cache.shape != v_cache.shape:
+        raise ValueError("q must be [B, H, T, d] and the caches [B, Hkv, W, d]")
+    B, H, T, d = q.shape
+    if k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError("cache shape does not match q")
+    Hkv, W = k_cache.shape[1], k_cache.shape[2]
+    if pos.dtype != torch.int32 or pos.shape != (B,) or not pos.is_cuda or not pos.is_contiguous():
+        raise ValueError("pos must be a contiguous int32 CUDA tensor [B]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_multi_workspace_bytes(B, H, Hkv, T, W, window, d), dtype=torch.uint8,
+                                device=q.device)
+    with torch.cuda.device(q.device):
+        rc = lib().attn_decode_multi(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), pos.data_ptr(),
+                                     out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), B, H, Hkv, T, W, int(window), d,
+                                     float(scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_decode_multi")
     return out, lse
 
 

@@ -185,9 +185,10 @@ BLOCK_N16384 = Workload("B2-H16-n16384-d128-block512", 2, 16, 16384, 128, False,
 
 @dataclasses.dataclass(frozen=True)
 class DecodeWorkload:
-    """One decode step against rolling key/value caches of W slots: one query
-    token per sequence at position `pos` (every sequence at the same
-    position), grouped-query heads."""
+    """One decode step against rolling key/value caches of W slots: T new
+    query tokens per sequence, the last at position `pos` (every sequence at
+    the same position), grouped-query heads, causal window `window` per token
+    (-1: W - 1, the whole cache)."""
 
     name: str
     B: int
@@ -198,20 +199,33 @@ class DecodeWorkload:
     pos: int
     q_std: float = 1.0
     seed: int = 0
+    T: int = 1
+    window: int = -1
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     @property
+    def w(self) -> int:
+        return self.W - 1 if self.window < 0 else self.window
+
+    @property
     def keys(self) -> int:
-        """Cached positions each query attends to."""
+        """Cached positions the step reads (every cached slot)."""
         return min(self.pos + 1, self.W)
+
+    @property
+    def attended(self) -> int:
+        """Attended (token, position) pairs per query head: token u at
+        position pos - T + 1 + u sees min(t_u, w) + 1 positions."""
+        return sum(min(self.pos - self.T + 1 + u, self.w) + 1 for u in range(self.T))
 
     def describe(self) -> dict:
         return {"workload": self.name, "B": self.B, "H": self.H, "H_kv": self.Hkv, "cache_slots": self.W,
-                "d": self.d, "position": self.pos, "keys_per_query": self.keys,
-                "scale": f"1/sqrt({self.d})", "q_std": self.q_std, "seed": self.seed}
+                "d": self.d, "tokens_per_sequence": self.T, "window": self.w, "position": self.pos,
+                "cached_positions_read": self.keys, "scale": f"1/sqrt({self.d})", "q_std": self.q_std,
+                "seed": self.seed}
 
 
 def make_decode(B: int, H: int, Hkv: int, W: int, d: int, seed: int = 0, q_std: float = 1.0
@@ -221,6 +235,20 @@ def make_decode(B: int, H: int, Hkv: int, W: int, d: int, seed: int = 0, q_std: 
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     q = torch.randn((B, H, d), generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q.mul_(q_std)
+    k = torch.randn((B, Hkv, W, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, W, d), generator=g, dtype=torch.float32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def make_decode_multi(B: int, H: int, Hkv: int, T: int, W: int, d: int, seed: int = 0, q_std: float = 1.0
+                      ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """q [B, H, T, d] and rolling caches k, v [B, Hkv, W, d], bf16, drawn like
+    make_decode (q, then k, then v from one generator seeded `seed`)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((B, H, T, d), generator=g, dtype=torch.float32)
     if q_std != 1.0:
         q.mul_(q_std)
     k = torch.randn((B, Hkv, W, d), generator=g, dtype=torch.float32)
@@ -242,10 +270,17 @@ def ring_from_sequence(seq: torch.Tensor, W: int) -> torch.Tensor:
 # worked example's cache size), Mistral-7B-like heads (32 query heads sharing
 # 8 key/value heads, d = 128), 64 sequences per step.
 DECODE_W4096 = DecodeWorkload("decode-B64-H32-Hkv8-W4096-d128-pos32767", 64, 32, 8, 4096, 128, 32767)
+# The same caches with four new tokens per sequence (a speculative step): the
+# 4096-slot cache serves a window of 4092 earlier positions to each of them.
+DECODE_T4_W4096 = DecodeWorkload("decode-B64-H32-Hkv8-T4-W4096-w4092-d128-pos32767", 64, 32, 8, 4096, 128,
+                                 32767, T=4, window=4092)
 
 
 def decode_by_name(name: str) -> Optional[DecodeWorkload]:
-    return DECODE_W4096 if name == DECODE_W4096.name else None
+    for wl in (DECODE_W4096, DECODE_T4_W4096):
+        if wl.name == name:
+            return wl
+    return None
 
 
 def sweep() -> List[Workload]:

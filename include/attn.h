@@ -305,7 +305,7 @@ ATTN_API int64_t attn_bwd_workspace_bytes(int B, int H, int n, int d);
  *   workspace        : device scratch owned by the caller, 16-byte aligned,
  *                      at least attn_decode_workspace_bytes(...) bytes
  *                      (per-split partial results)
- *   H / Hkv          : 1, 2, 4 or 8 (else ATTN_ERR_UNSUPPORTED); d: 64 or 128
+ *   H / Hkv          : 1 .. 16 (else ATTN_ERR_UNSUPPORTED); d: 64 or 128
  *   B * Hkv          : at most 65535
  *   scale, stream    : as attn_fwd
  *
@@ -324,6 +324,53 @@ ATTN_API int attn_decode(const void *q, const void *k_cache, const void *v_cache
 /* Device workspace bytes attn_decode needs, or -1 if the shape is invalid
  * or unsupported. */
 ATTN_API int64_t attn_decode_workspace_bytes(int B, int H, int Hkv, int W, int d);
+
+/*
+ * attn_decode_multi - a decode step with a few new query tokens per sequence
+ * (speculative decoding, chunked steps) against rolling key/value caches.
+ *
+ * Every sequence b has T new tokens at positions t_u = pos[b] - T + 1 + u,
+ * u = 0 .. T-1 (pos[b], >= T - 1, is the last of them), and their keys and
+ * values have already been written to the rolling cache of W slots
+ * (position p in slot p mod W; the rolling buffer of "Beyond attention",
+ * section "For engineers -- Show the maths"). Token u attends causally: to
+ * the positions max(0, t_u - window) .. t_u of its sliding window (the
+ * causal window-w mask of "week17 efficiency attention", local attention
+ * section), so the T outputs are rows t_0 .. t_{T-1} of attn_fwd with
+ * causal = 1 and window = `window` over the sequence that filled the cache:
+ *
+ *   O[b,h,u]   = softmax(scale * q[b,h,u] . k) v   over that window,
+ *   LSE[b,h,u] = ln sum exp(scale * q[b,h,u] . k)  (natural-log units),
+ *
+ * with key/value head h / (H / Hkv). A W-slot cache still holds every
+ * position of every token's window when window + T <= W; other windows give
+ * ATTN_ERR_INVALID. attn_decode is the case T = 1, window = W - 1.
+ *
+ *   q                : device, bf16 [B, H, T, d], 16-byte aligned
+ *   k_cache, v_cache : device, bf16 [B, Hkv, W, d], 16-byte aligned, read only
+ *   pos              : device, int32 [B] (a value below T - 1 is read as T - 1)
+ *   o, lse           : device, bf16 [B, H, T, d] and fp32 [B, H, T], written
+ *   workspace        : device scratch owned by the caller, 16-byte aligned, at
+ *                      least attn_decode_multi_workspace_bytes(...) bytes
+ *   (H / Hkv) * T    : at most 16 (the query rows of one key/value head fill
+ *                      one 16-wide MMA), else ATTN_ERR_UNSUPPORTED
+ *   B, Hkv, d, scale, stream : as attn_decode
+ *
+ * The step reads every cached slot (W slots once the cache is full), also
+ * those that only lie outside every token's window when window + T < W;
+ * size the cache W = window + T to read no slot in vain. Slots no position
+ * has reached yet may hold any bits, NaN included. Arithmetic, kernels and
+ * return values as attn_decode.
+ */
+ATTN_API int attn_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                               const int *pos, void *o, float *lse, void *workspace,
+                               size_t workspace_bytes, int B, int H, int Hkv, int T, int W,
+                               int window, int d, float scale, void *stream);
+
+/* Device workspace bytes attn_decode_multi needs, or -1 if the arguments are
+ * invalid or unsupported. */
+ATTN_API int64_t attn_decode_multi_workspace_bytes(int B, int H, int Hkv, int T, int W, int window,
+                                                   int d);
 
 /*
  * attn_sync_status - synchronize `stream`, then read and clear this device's

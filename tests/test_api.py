@@ -173,7 +173,7 @@ def test_bwd_binding_checks_tensors_before_calling(attn):
 @pytest.mark.parametrize("kw,code", [
     (dict(q=0), 1), (dict(pos=0), 1), (dict(workspace=0), 1), (dict(B=0), 1), (dict(W=0), 1),
     (dict(scale=0.0), 1), (dict(Hkv=3), 1), (dict(q=FAKE + 8), 1), (dict(pos=FAKE + 2), 1),
-    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(H=24, Hkv=2), 2), (dict(H=16, Hkv=1), 2),
+    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(H=34, Hkv=2), 2), (dict(H=32, Hkv=1), 2),
     (dict(B=70000, H=8, Hkv=1), 2),
 ])
 def test_attn_decode_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
@@ -203,7 +203,29 @@ def test_decode_workspace_size(attn):
         return ((W + chunk - 1) // chunk) * B * H * (d + 2) * 4
     for shape in [(1, 1, 1, 1, 64), (2, 8, 2, 4096, 128), (64, 32, 8, 4096, 128), (3, 4, 4, 200, 64)]:
         assert attn.decode_workspace_bytes(*shape) == expect(*shape)
-    assert attn.lib().attn_decode_workspace_bytes(1, 6, 2, 64, 64) == -1
+    assert attn.lib().attn_decode_workspace_bytes(1, 34, 2, 64, 64) == -1  # 17 query heads per K/V head
+    # several new tokens per sequence: T partial rows per (b, h)
+    for B, H, Hkv, T, W, w, d in [(2, 8, 2, 4, 4096, 4092, 128), (64, 32, 8, 4, 4096, 4092, 128),
+                                  (3, 6, 2, 3, 200, 50, 64), (1, 16, 1, 1, 128, 127, 64)]:
+        assert attn.decode_multi_workspace_bytes(B, H, Hkv, T, W, w, d) == expect(B, H, Hkv, W, d) * T
+    # T = 1 with the whole cache as the window is attn_decode
+    assert attn.decode_multi_workspace_bytes(2, 8, 2, 1, 4096, 4095, 128) == attn.decode_workspace_bytes(
+        2, 8, 2, 4096, 128)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=0), 1), (dict(window=-1), 1), (dict(window=4093), 1), (dict(T=5, window=4092), 1),
+    (dict(H=20, Hkv=5, T=5, window=100), 2), (dict(H=8, Hkv=1, T=3, window=100), 2), (dict(q=0), 1),
+    (dict(ws_bytes=0), 1), (dict(d=96), 2), (dict(Hkv=3), 1),
+])
+def test_attn_decode_multi_rejects_bad_arguments_before_any_cuda_call(attn, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, pos=FAKE, o=FAKE, lse=FAKE, workspace=FAKE, ws_bytes=1 << 40,
+             B=2, H=8, Hkv=2, T=4, W=4096, window=4092, d=128, scale=0.125, stream=None)
+    a.update(kw)
+    rc = attn.lib().attn_decode_multi(a["q"], a["k"], a["v"], a["pos"], a["o"], a["lse"], a["workspace"],
+                                      a["ws_bytes"], a["B"], a["H"], a["Hkv"], a["T"], a["W"], a["window"],
+                                      a["d"], a["scale"], a["stream"])
+    assert rc == code
 
 
 def test_bwd_gqa_entry_point_rejects_bad_head_counts(attn):
