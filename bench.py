@@ -456,6 +456,7 @@ def run_ours(args, wl, world, rank, local):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": args.steps,
+        "fwd_schedule": args.schedule,
         "clocks": clocks.summary(wall0, wall1),
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -721,7 +722,7 @@ def run_sweep(args):
             times.append(a.elapsed_time(b))
         ms = statistics.median(times)
         tf = flops / (ms / 1e3) / 1e12
-        print(json.dumps({"workload": wl.name, "ms": ms, "tflops": tf,
+        print(json.dumps({"workload": wl.name, "schedule": args.schedule, "ms": ms, "tflops": tf,
                           "pct_of_peak": 100 * tf / bf16_peak, "hbm_gbs": min_bytes / (ms / 1e3) / 1e9,
                           "pct_of_hbm": 100 * min_bytes / (ms / 1e3) / 1e9 / hbm_peak,
                           "status": st, "l2": "flushed (256 MB write) before each timed launch",
@@ -751,12 +752,18 @@ def main():
                          "sequence (attn_decode_multi)")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (attn_bwd) of --workload instead of the forward")
+    ap.add_argument("--schedule", choices=["auto", "per_item", "persistent"], default="auto",
+                    help="forward work schedule (attn_fwd_schedule): automatic by mask and length, or forced")
     ap.add_argument("--profile", action="store_true",
                     help="timed kernel launches only (no e2e, CPU baseline or clock sampling): "
                          "the command profiled under ncu")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.schedule != "auto" and args.impl == "ours":
+        import exact_softmax_attention_04_b200 as attn
+        attn.set_fwd_schedule({"per_item": attn.SCHEDULE_PER_ITEM,
+                               "persistent": attn.SCHEDULE_PERSISTENT}[args.schedule])
     if args.sweep:
         return run_sweep(args)
     from exact_softmax_attention_04_b200 import synth

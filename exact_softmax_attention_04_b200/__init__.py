@@ -31,7 +31,7 @@ EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_relea
            "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
            "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes", "attn_decode",
            "attn_decode_workspace_bytes", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
-           "attn_fwd_blocklocal", "attn_bwd_blocklocal")
+           "attn_fwd_blocklocal", "attn_bwd_blocklocal", "attn_fwd_schedule")
 
 
 class AttnError(RuntimeError):
@@ -86,6 +86,8 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_decode.restype = i
     lib.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.attn_decode_workspace_bytes.restype = i64
+    lib.attn_fwd_schedule.argtypes = [i]
+    lib.attn_fwd_schedule.restype = i
     lib.attn_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, i, i, f, vp]
     lib.attn_decode_multi.restype = i
     lib.attn_decode_multi_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
@@ -286,6 +288,18 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, p
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_decode")
     return out, lse
+
+
+SCHEDULE_AUTO, SCHEDULE_PER_ITEM, SCHEDULE_PERSISTENT = 0, 1, 2
+
+
+def set_fwd_schedule(mode: int) -> int:
+    """Process-wide forward work schedule (auto / one CTA per work item /
+    persistent); returns the previous mode. See attn_fwd_schedule."""
+    prev = int(lib().attn_fwd_schedule(int(mode)))
+    if prev < 0:
+        raise ValueError(f"unknown schedule {mode}")
+    return prev
 
 
 def decode_multi_workspace_bytes(B: int, H: int, Hkv: int, T: int, W: int, window: int, d: int) -> int:

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -90,7 +92,8 @@ namespace {
 
 using namespace attn_host;
 
-bool g_smem_set[kMaxDevices][2][2] = {};  // [device][d==128][block mask]
+bool g_smem_set[kMaxDevices][2][2][2] = {};  // [device][d==128][block mask][persistent]
+int g_num_sms[kMaxDevices] = {};
 
 struct Staging {
     void *buf = nullptr;
@@ -163,27 +166,74 @@ int check_args(const void *q, const void *k, const void *v, const void *o, const
 
 // Sets the kernel's launch attributes once per device and checks its
 // register count against the split it was compiled for.
-template <int D, bool BLOCKMASK>
+template <int D, bool BLOCKMASK, bool PERSIST>
 int prepare_fwd(int dev)
 {
     using Cfg = attn_sm100::FwdCfg<D>;
     std::lock_guard<std::mutex> lk(g_mu);
-    bool &set = g_smem_set[dev][D == 128 ? 1 : 0][BLOCKMASK ? 1 : 0];
+    bool &set = g_smem_set[dev][D == 128 ? 1 : 0][BLOCKMASK ? 1 : 0][PERSIST ? 1 : 0];
     if (set) return ATTN_OK;
+    if (!g_num_sms[dev] &&
+        (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+         g_num_sms[dev] <= 0))
+        return ATTN_ERR_CUDA;
     // The kernel moves registers between its warpgroups; that only works if it
     // is launched with exactly the per-thread register count the split was
     // computed for (else the raising warps wait forever). Refuse to launch a
     // build that differs.
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D, BLOCKMASK>) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST>) != cudaSuccess)
         return ATTN_ERR_CUDA;
     if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D, BLOCKMASK>,
+    if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
     set = true;
     return ATTN_OK;
+}
+
+// Persistent schedule or one CTA per work item, and the persistent form's
+// item order. Measured on one B200 over the target workloads (a sweep of
+// n = 1024 ... 65536, d = 64 and 128, five masks, plus the configurations):
+// - windows (and block masks) whose query tiles walk at most ~12 key tiles
+//   (w = 256 and 1024, symmetric window 256): persistent, head-major order,
+//   +3% to +29%; a CTA's set-up, Q load and epilogue are otherwise as long as
+//   its key loop. w = 4096: one CTA per item (2% to 6% faster);
+// - no mask: persistent only for short sequences (n <= 1536: +3% to +12%);
+//   long rows: one CTA per item (persistent 2% to 7% slower);
+// - causal without a window: persistent with pair-major items up to
+//   n = 16384 (+3% to +18%: the hardware's CTA dispatch handles the unequal
+//   causal items worse than the balanced snake), one CTA per item above
+//   (2% to 9% faster at n >= 65536).
+// ATTN_FWD_PERSIST_MAX_TILES (build time) moves the key-tile threshold; 0
+// disables the persistent form in the automatic choice.
+#ifndef ATTN_FWD_PERSIST_MAX_TILES
+#define ATTN_FWD_PERSIST_MAX_TILES 12
+#endif
+std::atomic<int> g_schedule{ATTN_SCHEDULE_AUTO};
+
+enum FwdSchedule { kPerItem = 0, kPersistHeadMajor = 1, kPersistPairMajor = 2 };
+
+// window and block as the kernels see them (effective_window/_block).
+FwdSchedule fwd_schedule(int n, int causal, int window, int block)
+{
+    const bool causal_only = causal && window < 0 && block <= 0;
+    const FwdSchedule persist = causal_only ? kPersistPairMajor : kPersistHeadMajor;
+    const int mode = g_schedule.load(std::memory_order_relaxed);
+    if (mode == ATTN_SCHEDULE_PERSISTENT) return persist;
+    if (mode == ATTN_SCHEDULE_PER_ITEM || ATTN_FWD_PERSIST_MAX_TILES <= 0) return kPerItem;
+    if (causal_only) return n <= 16384 ? kPersistPairMajor : kPerItem;
+    double keys;  // about the keys a query row attends to
+    if (block > 0)
+        keys = causal ? 1.5 * block : 2.0 * block;
+    else if (window >= 0)
+        keys = causal ? window : 2.0 * window;
+    else
+        keys = n;
+    const double q_tiles = (n + attn_sm100::BM - 1) / attn_sm100::BM;
+    const double tiles = std::min(q_tiles, keys / attn_sm100::BN + 2.0);
+    return tiles <= ATTN_FWD_PERSIST_MAX_TILES ? kPersistHeadMajor : kPerItem;
 }
 
 template <int D>
@@ -202,9 +252,8 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
         !encode_bhnd(enc, &mv, v, bhkv, n, D) || !encode_bhnd(enc, &mo, o, bh, n, D))
         return ATTN_ERR_CUDA;
     const bool blockmask = effective_block(n, block) > 0;
-    const int prc = blockmask ? prepare_fwd<D, true>(dev) : prepare_fwd<D, false>(dev);
-    if (prc != ATTN_OK) return prc;
     attn_sm100::FwdParams p;
+    p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.status = status;
     p.heads = H;
@@ -216,15 +265,37 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     p.causal = causal;
     p.window = effective_window(n, window);
     p.block = effective_block(n, block);
-    const unsigned grid = static_cast<unsigned>(bh * p.num_cta_tiles);
+    p.num_work = static_cast<int>(bh * p.num_cta_tiles);
+    const FwdSchedule sched = fwd_schedule(n, causal, p.window, p.block);
+    const bool persist = sched != kPerItem;
+    p.pair_major = sched == kPersistPairMajor ? 1 : 0;
+    int prc = ATTN_OK;
     if (blockmask)
-        attn_sm100::attn_fwd_kernel<D, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        prc = persist ? prepare_fwd<D, true, true>(dev) : prepare_fwd<D, true, false>(dev);
     else
-        attn_sm100::attn_fwd_kernel<D, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        prc = persist ? prepare_fwd<D, false, true>(dev) : prepare_fwd<D, false, false>(dev);
+    if (prc != ATTN_OK) return prc;
+    const unsigned grid = static_cast<unsigned>(persist ? std::min(p.num_work, g_num_sms[dev]) : p.num_work);
+    using namespace attn_sm100;
+    if (blockmask && persist)
+        attn_fwd_kernel<D, true, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else if (blockmask)
+        attn_fwd_kernel<D, true, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else if (persist)
+        attn_fwd_kernel<D, false, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else
+        attn_fwd_kernel<D, false, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace
+
+extern "C" int attn_fwd_schedule(int mode)
+{
+    if (mode != ATTN_SCHEDULE_AUTO && mode != ATTN_SCHEDULE_PER_ITEM && mode != ATTN_SCHEDULE_PERSISTENT)
+        return -1;
+    return g_schedule.exchange(mode);
+}
 
 extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                         int H, int n, int d, float scale, int causal, int window, void *stream)

@@ -101,6 +101,28 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
              void *stream);
 
 /*
+ * attn_fwd_schedule - how the forward kernels (attn_fwd, attn_fwd_gqa,
+ * attn_fwd_blocklocal and the host-buffer forms) spread their work over the
+ * SMs; a process-wide setting for tuning and testing, read at each launch.
+ *
+ *   ATTN_SCHEDULE_AUTO       : by the mask and n (the default): the
+ *                              persistent form when a query tile walks few
+ *                              key tiles on average, else one CTA per item
+ *   ATTN_SCHEDULE_PER_ITEM   : one CTA per work item (two 128-row query
+ *                              tiles of one head)
+ *   ATTN_SCHEDULE_PERSISTENT : one CTA per SM walking the work items
+ *
+ * Both forms compute the same result bit for bit (the same arithmetic per
+ * tile in the same order). Returns the previous mode, or -1 (and changes
+ * nothing) for an unknown mode. Not synchronised with launches in flight on
+ * other threads: set it before enqueueing work.
+ */
+#define ATTN_SCHEDULE_AUTO 0
+#define ATTN_SCHEDULE_PER_ITEM 1
+#define ATTN_SCHEDULE_PERSISTENT 2
+ATTN_API int attn_fwd_schedule(int mode);
+
+/*
  * attn_fwd_gqa - grouped-query (and multi-query) attention on device buffers.
  *
  * Grouped-query attention ("week17 efficiency attention", MQA / GQA section):

@@ -254,3 +254,13 @@ def test_block_pair_count_workload(attn):
     wl = synth.BLOCK_N16384
     # 32 blocks of 512: block 0 sees itself (512 keys), later blocks 1024 keys
     assert synth.workload_pairs_per_head(wl) == 512 * 512 + 31 * 512 * 1024
+
+
+def test_fwd_schedule_setting(attn):
+    lib = attn.lib()
+    assert lib.attn_fwd_schedule(attn.SCHEDULE_PERSISTENT) == attn.SCHEDULE_AUTO
+    assert lib.attn_fwd_schedule(attn.SCHEDULE_PER_ITEM) == attn.SCHEDULE_PERSISTENT
+    assert lib.attn_fwd_schedule(7) == -1                      # unknown: nothing changes
+    assert lib.attn_fwd_schedule(attn.SCHEDULE_AUTO) == attn.SCHEDULE_PER_ITEM
+    with pytest.raises(ValueError):
+        attn.set_fwd_schedule(-3)

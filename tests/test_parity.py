@@ -59,13 +59,59 @@ MASKS = [(False, -1), (True, -1), (True, 0), (True, 1), (True, 127), (True, 128)
          (True, 300), (True, 100000), (False, 0), (False, 1), (False, 127), (False, 200), (False, 100000)]
 
 
+@pytest.fixture(params=["per_item", "persistent"])
+def schedule(request, attn):
+    """Run the test under one forward work schedule (forced), then restore
+    the automatic choice."""
+    mode = {"per_item": attn.SCHEDULE_PER_ITEM, "persistent": attn.SCHEDULE_PERSISTENT}[request.param]
+    attn.set_fwd_schedule(mode)
+    yield request.param
+    attn.set_fwd_schedule(attn.SCHEDULE_AUTO)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("n", [1, 77, 128, 129, 256, 383, 640])
 @pytest.mark.parametrize("causal,window", MASKS)
-def test_small_shapes_all_masks_in_full(attn, oracle_mod, d, n, causal, window):
+def test_small_shapes_all_masks_in_full(attn, oracle_mod, schedule, d, n, causal, window):
     q_std = 4.0 if (n + d + window) % 2 else 1.0
     q, k, v = synth.make_qkv(1, 2, n, d, seed=n * 7 + d, q_std=q_std)
-    _full_check(attn, oracle_mod, q, k, v, causal, window, what=f"n{n} d{d} c{causal} w{window}")
+    _full_check(attn, oracle_mod, q, k, v, causal, window, what=f"{schedule} n{n} d{d} c{causal} w{window}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,H,Hkv,n,causal,window,block", [
+    (3, 5, 5, 700, True, 200, 0), (2, 8, 2, 1000, True, -1, 0), (1, 6, 3, 2100, False, 300, 0),
+    (2, 4, 4, 1500, False, -1, 0), (1, 8, 8, 3000, True, -1, 512), (2, 4, 1, 999, False, -1, 256)])
+def test_schedules_agree_bit_for_bit(attn, d, B, H, Hkv, n, causal, window, block):
+    """The persistent form walks the same work items with the same per-tile
+    arithmetic as one CTA per item: equal outputs, bit for bit (many items
+    per persistent CTA here: grouped heads, block masks, ragged tails)."""
+    q, k, v = synth.make_qkv(B, H, n, d, seed=B * 100 + n + d, q_std=3.0, Hkv=Hkv)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    outs = []
+    try:
+        for mode in (attn.SCHEDULE_PER_ITEM, attn.SCHEDULE_PERSISTENT):
+            attn.set_fwd_schedule(mode)
+            o, lse = attn.attn_fwd(qd, kd, vd, None, causal, window, block=block)
+            assert attn.sync_status() == attn.ATTN_OK
+            outs.append((o, lse))
+    finally:
+        attn.set_fwd_schedule(attn.SCHEDULE_AUTO)
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_persistent_schedule_many_items_per_cta(attn, oracle_mod):
+    """64 heads x 24 query-tile pairs = 1536 items over the SMs (about ten per
+    persistent CTA), window 256, both head sizes; sampled rows against the
+    oracle."""
+    try:
+        attn.set_fwd_schedule(attn.SCHEDULE_PERSISTENT)
+        for d in (64, 128):
+            wl = synth.Workload(f"persist-B4-H16-n6000-d{d}-window256", 4, 16, 6000, d, True, 256, q_std=4.0)
+            rows = synth.sample_rows(wl.B, wl.H, wl.n, per_head_random=64, seed=5)
+            _sampled_check(attn, oracle_mod, wl, rows)
+    finally:
+        attn.set_fwd_schedule(attn.SCHEDULE_AUTO)
 
 
 def test_batch_and_many_heads(attn, oracle_mod):
