@@ -118,8 +118,8 @@ struct FwdCfg {
     static constexpr int KV_OFF = Q_OFF + QT * TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
     // q_full[QT], kv_full[NSLOT], kv_empty[NSLOT], s_full[QT], p_full[QT], o_done[QT],
-    // s_free[QT], pv_done[QT], q_empty[QT], o_free[QT], drain
-    static constexpr int NUM_BARS = QT + 2 * NSLOT + 7 * QT + 1;
+    // s_free[QT], pv_done[QT], o_free[QT], q_empty[QT], drain[QT]
+    static constexpr int NUM_BARS = 2 * QT + 2 * NSLOT + 7 * QT;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + 1 KB alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -370,9 +370,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     auto o_done = [&](int s) { return bars + 8u * (3 * QT + 2 * NSLOT + s); };
     auto s_free = [&](int s) { return bars + 8u * (4 * QT + 2 * NSLOT + s); };
     auto pv_done = [&](int s) { return bars + 8u * (5 * QT + 2 * NSLOT + s); };
-    auto q_empty = [&](int s) { return bars + 8u * (6 * QT + 2 * NSLOT + s); };
-    auto o_free = [&](int s) { return bars + 8u * (7 * QT + 2 * NSLOT + s); };
-    const uint32_t drain_bar = bars + 8u * (8 * QT + 2 * NSLOT);
+    auto o_free = [&](int s) { return bars + 8u * (6 * QT + 2 * NSLOT + s); };
+    auto q_empty = [&](int s) { return bars + 8u * (7 * QT + 2 * NSLOT + s); };
+    auto drain_bar = [&](int s) { return bars + 8u * (8 * QT + 2 * NSLOT + s); };
+    // The persistent form gives each query-tile slot an MMA issuer of its own
+    // (warp 8: slot 0, warp 10: slot 1), so that one slot's walk over its key
+    // tiles and items never waits for the other's: with a window the two
+    // tiles of an item walk key ranges one tile apart, and with one issuer
+    // the next item's first S waited for the later tile's last PV.
+    constexpr bool DUAL = PERSIST;
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
@@ -391,14 +397,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             mbar_init(o_done(s), 1);
             mbar_init(s_free(s), BM);
             mbar_init(pv_done(s), 1);
-            mbar_init(q_empty(s), 1);
             mbar_init(o_free(s), BM);
+            mbar_init(q_empty(s), 1);
         }
         for (int i = 0; i < NSLOT; ++i) {
             mbar_init(kv_full(i), 1);
-            mbar_init(kv_empty(i), 1);
+            mbar_init(kv_empty(i), DUAL ? QT : 1);  // one release per issuing warp
         }
-        mbar_init(drain_bar, 1);
+        for (int s = 0; s < QT; ++s) mbar_init(drain_bar(s), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -478,7 +484,113 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             for (int slot = 0; slot < NSLOT; ++slot)
                 if (item > slot) wt.drain(kv_full(slot), ((item - 1 - slot) / NSLOT) & 1u);
         }
-      } else if (warp == 8) {
+      } else if (DUAL && (warp == 8 || warp == 10)) {
+        // ------------------------------------------------------------ MMA issuers, one per slot
+        // Both walk every key tile of every item and release each ring slot
+        // (kv_empty counts one release per warp), after waiting for the slot
+        // to fill, also when their tile does not use it: so neither can
+        // release a slot's next use before the other has released this one.
+        const int s = (warp == 10) ? 1 : 0;
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+        const uint64_t kdesc0 = smem_desc_sw128(sKV(0), 16, 1024);
+        const uint64_t vdesc0 = smem_desc_sw128(sKV(0), BOX_BYTES, 1024);
+        const uint32_t s_col = tmem + C::S_COL + s * BN;
+        const uint32_t o_col = tmem + C::O_COL + s * D;
+        const uint32_t p_col = tmem + C::P_COL + s * C::P_STRIDE;
+        int qn = 0, sn = 0, pn = 0, tn = 0;  // Q tiles, S and PV MMAs, items of this slot
+        int item = 0;                        // ring items walked
+        bool issued = false;                 // any MMA issued by this warp yet
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int w = fwd_item<PERSIST>(p, it);
+            if (w == -2) break;
+            if (w < 0) continue;
+            const FwdWork t = fwd_work<BLOCKMASK, PERSIST>(p, w);
+            const int my_lo = s ? t.jlo_s[1] : t.jlo_s[0], my_hi = s ? t.jhi_s[1] : t.jhi_s[0];
+            if (my_hi > my_lo) {
+                ok = __all_sync(0xffffffffu, wt.wait(q_full(s), qn & 1u));
+                ++qn;
+            }
+            tc_fence_after();
+            const uint64_t qdesc = smem_desc_sw128(sQ(s), 16, 1024);
+            const int item0 = item;
+            for (int j = t.jlo; ok && j <= t.jhi; ++j) {
+                const int ik = item0 + 2 * (j - t.jlo);
+                const int iv = ik - 1;
+                if (j < t.jhi && !__all_sync(0xffffffffu, wt.wait(kv_full(ik % NSLOT), (ik / NSLOT) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                if (j > t.jlo && !__all_sync(0xffffffffu, wt.wait(kv_full(iv % NSLOT), (iv / NSLOT) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t kdesc = kdesc0 + static_cast<uint64_t>(((ik % NSLOT) * C::TILE_BYTES) >> 4);
+                const uint64_t vdesc = vdesc0 + static_cast<uint64_t>(((iv % NSLOT) * C::TILE_BYTES) >> 4);
+                auto issue_pv = [&]() -> bool {
+                    const bool first = (j - 1 == my_lo);
+                    if (!__all_sync(0xffffffffu, wt.wait(p_full(s), pn & 1u))) return false;
+                    if (first && tn > 0 && !__all_sync(0xffffffffu, wt.wait(o_free(s), (tn - 1) & 1u)))
+                        return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < BN / 16; ++k)
+                        mma_bf16_ts_if(leader, o_col, p_col + k * 8, vdesc + static_cast<uint64_t>(k * 128),
+                                       idesc_pv, (!first || k > 0) ? 1u : 0u);
+                    ++pn;
+                    if constexpr (C::SPLIT_P) mma_commit_if(leader, pv_done(s));
+                    if (j == my_hi) {
+                        mma_commit_if(leader, o_done(s));
+                        ++tn;
+                    }
+                    return true;
+                };
+                auto issue_s = [&]() -> bool {
+                    if constexpr (C::SPLIT_P) {
+                        if (sn > 0 && !__all_sync(0xffffffffu, wt.wait(s_free(s), (sn - 1) & 1u))) return false;
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint64_t off = static_cast<uint64_t>(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                        mma_bf16_ss_if(leader, s_col, qdesc + off, kdesc + off, idesc_qk, k > 0 ? 1u : 0u);
+                    }
+                    mma_commit_if(leader, s_full(s));
+                    ++sn;
+                    if (j == my_hi - 1) mma_commit_if(leader, q_empty(s));
+                    return true;
+                };
+                const bool use_s = j >= my_lo && j < my_hi;
+                const bool use_pv = j - 1 >= my_lo && j - 1 < my_hi;
+                if constexpr (C::SPLIT_P) {
+                    if (use_s) ok = issue_s();
+                    if (ok && use_pv) ok = issue_pv();
+                } else {
+                    if (use_pv) ok = issue_pv();
+                    if (ok && use_s) ok = issue_s();
+                }
+                if (!ok) break;
+                issued = issued || use_s || use_pv;
+                // Release the slots once this warp's MMAs reading them are
+                // done (a commit tracks every MMA this warp has issued);
+                // before its first MMA, a plain arrive.
+                if (issued) {
+                    if (j < t.jhi) mma_commit_if(leader, kv_empty(ik % NSLOT));
+                    if (j > t.jlo) mma_commit_if(leader, kv_empty(iv % NSLOT));
+                } else {
+                    if (j < t.jhi && leader) mbar_arrive(kv_empty(ik % NSLOT));
+                    if (j > t.jlo && leader) mbar_arrive(kv_empty(iv % NSLOT));
+                }
+            }
+            item = item0 + 2 * (t.jhi - t.jlo);
+        }
+        if (issued) {
+            mma_commit_if(leader, drain_bar(s));
+            wt.drain(drain_bar(s), 0);
+        }
+      } else if (!DUAL && warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs this loop (uniform operands); one lane issues
         // every MMA and commit, so the commits track all of its MMAs.
@@ -592,8 +704,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             item = item0 + 2 * (t.jhi - t.jlo);
         }
         // Every MMA this warp issued must finish before TMEM is freed.
-        mma_commit_if(leader, drain_bar);
-        wt.drain(drain_bar, 0);
+        mma_commit_if(leader, drain_bar(0));
+        wt.drain(drain_bar(0), 0);
       }
     } else {
         // ------------------------------------------------------------ softmax
