@@ -456,7 +456,8 @@ def run_ours(args, wl, world, rank, local):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": args.steps,
-        "fwd_schedule": args.schedule,
+        "fwd_schedule": {"setting": args.schedule,
+                         "form": attn.fwd_schedule_for(wl.n, wl.causal, wl.window, wl.block)},
         "clocks": clocks.summary(wall0, wall1),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -31,7 +31,7 @@ EXPORTS = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_host", "attn_host_staging_relea
            "attn_sync_status", "attn_strerror", "attn_attended_pairs", "attn_fwd_host_noalloc",
            "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes", "attn_decode",
            "attn_decode_workspace_bytes", "attn_decode_multi", "attn_decode_multi_workspace_bytes",
-           "attn_fwd_blocklocal", "attn_bwd_blocklocal", "attn_fwd_schedule")
+           "attn_fwd_blocklocal", "attn_bwd_blocklocal", "attn_fwd_schedule", "attn_fwd_schedule_for")
 
 
 class AttnError(RuntimeError):
@@ -88,6 +88,8 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.attn_decode_workspace_bytes.restype = i64
     lib.attn_fwd_schedule.argtypes = [i]
     lib.attn_fwd_schedule.restype = i
+    lib.attn_fwd_schedule_for.argtypes = [i, i, i, i]
+    lib.attn_fwd_schedule_for.restype = i
     lib.attn_decode_multi.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, i, i, i, i, i, i, i, f, vp]
     lib.attn_decode_multi.restype = i
     lib.attn_decode_multi_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
@@ -300,6 +302,15 @@ def set_fwd_schedule(mode: int) -> int:
     if prev < 0:
         raise ValueError(f"unknown schedule {mode}")
     return prev
+
+
+def fwd_schedule_for(n: int, causal: bool, window: int = -1, block: int = 0) -> str:
+    """'per_item' or 'persistent': the form the forward takes for this
+    problem under the current setting (see attn_fwd_schedule_for)."""
+    r = int(lib().attn_fwd_schedule_for(int(n), int(bool(causal)), int(window), int(block)))
+    if r < 0:
+        raise ValueError("n must be >= 1")
+    return "persistent" if r == SCHEDULE_PERSISTENT else "per_item"
 
 
 def decode_multi_workspace_bytes(B: int, H: int, Hkv: int, T: int, W: int, window: int, d: int) -> int:

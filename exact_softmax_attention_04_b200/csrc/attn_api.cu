@@ -297,6 +297,14 @@ extern "C" int attn_fwd_schedule(int mode)
     return g_schedule.exchange(mode);
 }
 
+extern "C" int attn_fwd_schedule_for(int n, int causal, int window, int block)
+{
+    if (n < 1) return -1;
+    const int w = effective_window(n, window), b = effective_block(n, block);
+    return fwd_schedule(n, causal ? 1 : 0, b > 0 ? -1 : w, b) == kPerItem ? ATTN_SCHEDULE_PER_ITEM
+                                                                          : ATTN_SCHEDULE_PERSISTENT;
+}
+
 extern "C" int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B,
                         int H, int n, int d, float scale, int causal, int window, void *stream)
 {

@@ -123,6 +123,15 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
 ATTN_API int attn_fwd_schedule(int mode);
 
 /*
+ * attn_fwd_schedule_for - the form the forward kernels would take for a
+ * problem of n tokens with this mask under the current setting:
+ * ATTN_SCHEDULE_PER_ITEM or ATTN_SCHEDULE_PERSISTENT (never AUTO); -1 for
+ * n < 1. causal, window and block as for attn_fwd / attn_fwd_blocklocal
+ * (block <= 0: no block mask). Reports only; launches nothing.
+ */
+ATTN_API int attn_fwd_schedule_for(int n, int causal, int window, int block);
+
+/*
  * attn_fwd_gqa - grouped-query (and multi-query) attention on device buffers.
  *
  * Grouped-query attention ("week17 efficiency attention", MQA / GQA section):

@@ -264,3 +264,24 @@ def test_fwd_schedule_setting(attn):
     assert lib.attn_fwd_schedule(attn.SCHEDULE_AUTO) == attn.SCHEDULE_PER_ITEM
     with pytest.raises(ValueError):
         attn.set_fwd_schedule(-3)
+
+
+def test_fwd_schedule_for_reports_the_automatic_choice(attn):
+    """Plain causal: persistent up to n = 16384; windows and no mask:
+    persistent when a query tile walks few key tiles; a forced setting wins."""
+    f = attn.fwd_schedule_for
+    assert f(131072, True) == "per_item"          # the largest target workload
+    assert f(16384, True) == "persistent"
+    assert f(65536, True) == "per_item"
+    assert f(8192, False) == "per_item"           # no mask, long rows
+    assert f(1024, False) == "persistent"         # no mask, short rows
+    assert f(65536, True, 256) == "persistent"    # narrow window
+    assert f(32768, True, 4096) == "per_item"     # wide window
+    assert f(4096, True, 4096) == "persistent"    # a window of n or more is plain causal
+    assert f(16384, False, 256) == "persistent"   # symmetric window 256
+    prev = attn.set_fwd_schedule(attn.SCHEDULE_PERSISTENT)
+    try:
+        assert f(131072, True) == "persistent"
+    finally:
+        attn.set_fwd_schedule(prev)
+    assert attn.lib().attn_fwd_schedule_for(0, 1, -1, 0) == -1
