@@ -34,6 +34,10 @@
 // S_1(j). tcgen05 MMAs from one thread complete in issue order, so (a) S_s(j)
 // overwrites P_s(j-1) only after PV_s(j-1) has read it, and (b) when S_s(j)
 // is complete, PV_s(j-1) is too, so the softmax may rescale O_s right away.
+// With one CTA per item the softmax hands P_s over in two halves (keys 0..63,
+// then 64..127, each announced on its own barrier, O_s rescaled before the
+// first): the MMA warp issues PV_s on the first half while the softmax is
+// still computing the second.
 // D = 64: S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), S_s(j) waiting only until the
 // softmax has read S_s(j-1) into registers; the softmax waits for PV_s(j-1)
 // before it overwrites P_s or rescales O_s.
@@ -118,8 +122,8 @@ struct FwdCfg {
     static constexpr int KV_OFF = Q_OFF + QT * TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
     // q_full[QT], kv_full[NSLOT], kv_empty[NSLOT], s_full[QT], p_full[QT], o_done[QT],
-    // s_free[QT], pv_done[QT], o_free[QT], q_empty[QT], drain[QT]
-    static constexpr int NUM_BARS = 2 * QT + 2 * NSLOT + 7 * QT;
+    // s_free[QT], pv_done[QT], o_free[QT], q_empty[QT], drain[QT], p_half[QT]
+    static constexpr int NUM_BARS = 2 * QT + 2 * NSLOT + 8 * QT;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + 1 KB alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
@@ -142,6 +146,11 @@ struct FwdCfg {
     static constexpr int EX2_EMU = (D == 128) ? ATTN_EX2_EMU_D128 : ATTN_EX2_EMU_D64;
     static constexpr bool EMU_SPREAD = (D == 128);  // polynomial pairs spread along the row
     static constexpr bool MAX3 = (D == 128);        // row max with three-input max
+    // D = 128, one CTA per item: P handed over in two halves of 64 keys, the
+    // PV MMAs of the first half running while the softmax computes the
+    // second (measured +2% to +3%; slower in the persistent form, which
+    // keeps one hand-over).
+    static constexpr bool PV_SPLIT = (D == 128);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -373,12 +382,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     auto o_free = [&](int s) { return bars + 8u * (6 * QT + 2 * NSLOT + s); };
     auto q_empty = [&](int s) { return bars + 8u * (7 * QT + 2 * NSLOT + s); };
     auto drain_bar = [&](int s) { return bars + 8u * (8 * QT + 2 * NSLOT + s); };
+    auto p_half = [&](int s) { return bars + 8u * (9 * QT + 2 * NSLOT + s); };
     // The persistent form gives each query-tile slot an MMA issuer of its own
     // (warp 8: slot 0, warp 10: slot 1), so that one slot's walk over its key
     // tiles and items never waits for the other's: with a window the two
     // tiles of an item walk key ranges one tile apart, and with one issuer
     // the next item's first S waited for the later tile's last PV.
     constexpr bool DUAL = PERSIST;
+    constexpr bool PV_SPLIT = C::PV_SPLIT && !PERSIST;  // single issuer only
     uint32_t *const tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + C::MISC_OFF);
     volatile int *const abort_flag = reinterpret_cast<volatile int *>(base_ptr + C::MISC_OFF + 4);
 
@@ -394,6 +405,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             mbar_init(q_full(s), 1);
             mbar_init(s_full(s), 1);
             mbar_init(p_full(s), BM);
+            mbar_init(p_half(s), BM);
             mbar_init(o_done(s), 1);
             mbar_init(s_free(s), BM);
             mbar_init(pv_done(s), 1);
@@ -638,7 +650,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // O_s += P_s(j-1) V_{j-1}: BN/16 MMAs of 16 keys each
                 auto issue_pv = [&](int s) -> bool {
                     const bool first = (j - 1 == t.jlo_s[s]);
-                    if (!__all_sync(0xffffffffu, wt.wait(p_full(s), pn[s] & 1u))) return false;
+                    if (!__all_sync(0xffffffffu, wt.wait(PV_SPLIT ? p_half(s) : p_full(s), pn[s] & 1u)))
+                        return false;
                     // The first PV of an item overwrites O_s: the softmax must
                     // have read the previous item's O_s out.
                     if (first && tn[s] > 0 && !__all_sync(0xffffffffu, wt.wait(o_free(s), (tn[s] - 1) & 1u)))
@@ -647,9 +660,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     const uint32_t o_col = tmem + C::O_COL + s * D;
                     const uint32_t p_col = tmem + C::P_COL + s * C::P_STRIDE;
 #pragma unroll
-                    for (int k = 0; k < BN / 16; ++k)
+                    for (int k = 0; k < BN / 16; ++k) {
+                        // the second half of P_s once the softmax has stored it
+                        if (PV_SPLIT && k == BN / 32) {
+                            if (!__all_sync(0xffffffffu, wt.wait(p_full(s), pn[s] & 1u))) return false;
+                            tc_fence_after();
+                        }
                         mma_bf16_ts_if(leader, o_col, p_col + k * 8, vdesc + static_cast<uint64_t>(k * 128),
                                        idesc_pv, (!first || k > 0) ? 1u : 0u);
+                    }
                     ++pn[s];
                     if constexpr (C::SPLIT_P) mma_commit_if(leader, pv_done(s));
                     if (j == t.jhi_s[s]) {
@@ -828,10 +847,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // One straight-line body per case (no branch inside the unrolled
                 // loop, so MUFU and FMA work can be interleaved freely). Masked
                 // tiles always use the MUFU: the polynomial clamps at 2^-125.
-                auto exps = [&](auto emu) {
+                auto exps = [&](auto emu, auto i0, auto i1) {
                     constexpr int EMU = decltype(emu)::value;
 #pragma unroll
-                    for (int i = 0; i < BN / 2; ++i) {
+                    for (int i = decltype(i0)::value; i < decltype(i1)::value; ++i) {
                         const float2 x = ffma2(make_float2(u2f(sv[2 * i]), u2f(sv[2 * i + 1])), sc2, noff2);
                         float e0, e1;
                         if constexpr (EMU > 0) {
@@ -851,10 +870,58 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         pk[i] = pack_bf16x2(e0, e1);
                     }
                 };
-                if (C::EX2_EMU == 0 || need_mask)
-                    exps(std::integral_constant<int, 0>{});
+                using I0 = std::integral_constant<int, 0>;
+                using IH = std::integral_constant<int, BN / 4>;
+                using IE = std::integral_constant<int, BN / 2>;
+                const bool emu_off = (C::EX2_EMU == 0 || need_mask);
+                const bool do_rescale = u > 0 && __any_sync(0xffffffffu, rescale);
+                if constexpr (PV_SPLIT) {
+                    // First half of P (keys 0..63) -> TMEM; O_s rescaled; the
+                    // MMA warp may then run PV on that half while the second
+                    // half is computed.
+                    if (emu_off)
+                        exps(I0{}, I0{}, IH{});
+                    else
+                        exps(std::integral_constant<int, C::EX2_EMU>{}, I0{}, IH{});
+                    tmem_st32(p_base, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                    // O_s holds sum_{t<j} P_t V_t (PV_s(j-1) was issued before
+                    // S_s(j) and completed with it): rescale when a row's max grew.
+                    if (do_rescale) {
+                        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                        for (int h = 0; h < D / 64; ++h) {
+                            uint32_t o[64];
+                            tmem_ld64(o_base + h * 64, o);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const float2 v = fmul2(make_float2(u2f(o[2 * i]), u2f(o[2 * i + 1])), a2);
+                                o[2 * i] = f2u(v.x);
+                                o[2 * i + 1] = f2u(v.y);
+                            }
+                            tmem_st64(o_base + h * 64, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(p_half(s));
+                    if (emu_off)
+                        exps(I0{}, IH{}, IE{});
+                    else
+                        exps(std::integral_constant<int, C::EX2_EMU>{}, IH{}, IE{});
+                    tmem_st32(p_base + BN / 4, *reinterpret_cast<uint32_t(*)[32]>(&pk[BN / 4]));
+                    const float2 ps01 = fadd2(ps[0], ps[1]);
+                    const float2 ps23 = fadd2(ps[2], ps[3]);
+                    const float2 pst = fadd2(ps01, ps23);
+                    l = fmaf(l, alpha, pst.x + pst.y);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(p_full(s));
+                    continue;
+                }
+                if (emu_off)
+                    exps(I0{}, I0{}, IE{});
                 else
-                    exps(std::integral_constant<int, C::EX2_EMU>{});
+                    exps(std::integral_constant<int, C::EX2_EMU>{}, I0{}, IE{});
                 if constexpr (C::SPLIT_P) {
                     // P_s(j) reuses P_s(j-1)'s columns and O_s is about to be
                     // rescaled: PV_s(j-1) must be complete. (The first step of
@@ -875,7 +942,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // O_s holds sum_{t<j} P_t V_t: PV_s(j-1) has completed (waited for
                 // above with separate P buffers; otherwise it was issued before
                 // S_s(j) and completed with it). Rescale when a row's max grew.
-                if (u > 0 && __any_sync(0xffffffffu, rescale)) {
+                if (do_rescale) {
                     const float2 a2 = make_float2(alpha, alpha);
                     uint32_t o[D];
                     if constexpr (D == 128) tmem_ld128(o_base, o); else tmem_ld64(o_base, o);
