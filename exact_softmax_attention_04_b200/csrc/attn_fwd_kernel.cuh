@@ -41,9 +41,10 @@
 // D = 64: S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), S_s(j) waiting only until the
 // softmax has read S_s(j-1) into registers; the softmax waits for PV_s(j-1)
 // before it overwrites P_s or rescales O_s.
-// The exponentials run on the MUFU, and on unmasked tiles a fixed share of
-// them on the FMA pipe as a polynomial (see ex2_poly_x2); the share and the
-// form of the row max differ per head size (FwdCfg).
+// The exponentials run on the MUFU, and a fixed share of them on the FMA pipe
+// as a polynomial (see ex2_poly_x2): on every tile at d = 64, on unmasked
+// tiles at d = 128; the share and the form of the row max differ per head
+// size (FwdCfg).
 // Instantiations: BLOCKMASK = false for the causal and window masks (the
 // closed-form bounds), true for the block-local mask (Mask intervals); and
 // PERSIST: one CTA per work item (the pair of query tiles above), or one CTA
@@ -146,6 +147,11 @@ struct FwdCfg {
     static constexpr int EX2_EMU = (D == 128) ? ATTN_EX2_EMU_D128 : ATTN_EX2_EMU_D64;
     static constexpr bool EMU_SPREAD = (D == 128);  // polynomial pairs spread along the row
     static constexpr bool MAX3 = (D == 128);        // row max with three-input max
+    // Boundary (masked) tiles take the polynomial share too, their masked
+    // entries zeroed in P afterwards: at d = 64 +4% to +5% on causal
+    // workloads; at d = 128 the same cost 1% to 4%, so there they use the
+    // MUFU alone.
+    static constexpr bool EMU_MASKED = (D == 64);
     // D = 128, one CTA per item: P handed over in two halves of 64 keys, the
     // PV MMAs of the first half running while the softmax computes the
     // second (measured +2% to +3%; slower in the persistent form, which
@@ -784,14 +790,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                                  (!causal && window >= 0 && k0 + BN - 1 > q0 + window));
                 const bool mask_lo = BLOCKMASK ? (tile_first > k0) : (window >= 0 && k0 < q0 + BM - 1 - window);
                 const bool need_mask = mask_hi || mask_lo;
+                // Allowed keys of this row form one interval; in tile columns:
+                // [lo, hi] with key = k0 + column (on a side that cuts no row,
+                // the bound lies outside the tile).
+                const int hi = BLOCKMASK ? row_last - k0
+                                         : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
+                                               n - 1 - k0);
+                const int lo = BLOCKMASK ? row_first - k0 : ((window >= 0) ? row - window - k0 : 0);
                 if (need_mask) {
-                    // Allowed keys of this row form one interval; in tile columns:
-                    // [lo, hi] with key = k0 + column. Most masked tiles cut on
-                    // one side only, which takes one compare per element.
-                    const int hi = BLOCKMASK ? row_last - k0
-                                             : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
-                                                   n - 1 - k0);
-                    const int lo = BLOCKMASK ? row_first - k0 : ((window >= 0) ? row - window - k0 : 0);
+                    // Most masked tiles cut on one side only, which takes one
+                    // compare per element.
                     if (mask_hi && mask_lo) {
 #pragma unroll
                         for (int c = 0; c < BN; ++c)
@@ -845,8 +853,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 for (int i = 0; i < 4; ++i) ps[i] = make_float2(0.f, 0.f);
                 uint32_t pk[BN / 2];
                 // One straight-line body per case (no branch inside the unrolled
-                // loop, so MUFU and FMA work can be interleaved freely). Masked
-                // tiles always use the MUFU: the polynomial clamps at 2^-125.
+                // loop, so MUFU and FMA work can be interleaved freely). At
+                // d = 128 masked tiles use the MUFU alone.
                 auto exps = [&](auto emu, auto i0, auto i1) {
                     constexpr int EMU = decltype(emu)::value;
 #pragma unroll
@@ -873,7 +881,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 using I0 = std::integral_constant<int, 0>;
                 using IH = std::integral_constant<int, BN / 4>;
                 using IE = std::integral_constant<int, BN / 2>;
-                const bool emu_off = (C::EX2_EMU == 0 || need_mask);
+                const bool emu_off = (C::EX2_EMU == 0) || (!C::EMU_MASKED && need_mask);
+                // The polynomial clamps at 2^-125: on masked tiles the masked
+                // entries of its pairs are set to exactly 0 in P afterwards
+                // (the MUFU gives 0 for them by itself), so a masked key never
+                // reaches O, whatever its value. Their 2^-125 stays in the row
+                // sum l, below its rounding: from the first allowed key on, l
+                // holds the row maximum's 1.0 (and a tile with no allowed key
+                // before that is scaled away by alpha = 0).
+                auto fix_masked = [&](auto i0, auto i1) {
+                    if constexpr (C::EMU_MASKED && C::EX2_EMU > 0) {
+#pragma unroll
+                        for (int i = decltype(i0)::value; i < decltype(i1)::value; ++i) {
+                            if ((C::EMU_SPREAD ? ((i * C::EX2_EMU) % 16) : (i % 16)) < C::EX2_EMU) {
+                                const bool k0 = (2 * i >= lo) && (2 * i <= hi);
+                                const bool k1 = (2 * i + 1 >= lo) && (2 * i + 1 <= hi);
+                                pk[i] &= (k0 ? 0x0000FFFFu : 0u) | (k1 ? 0xFFFF0000u : 0u);
+                            }
+                        }
+                    }
+                };
                 const bool do_rescale = u > 0 && __any_sync(0xffffffffu, rescale);
                 if constexpr (PV_SPLIT) {
                     // First half of P (keys 0..63) -> TMEM; O_s rescaled; the
@@ -883,6 +910,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         exps(I0{}, I0{}, IH{});
                     else
                         exps(std::integral_constant<int, C::EX2_EMU>{}, I0{}, IH{});
+                    if (need_mask) fix_masked(I0{}, IH{});
                     tmem_st32(p_base, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
                     // O_s holds sum_{t<j} P_t V_t (PV_s(j-1) was issued before
                     // S_s(j) and completed with it): rescale when a row's max grew.
@@ -908,6 +936,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         exps(I0{}, IH{}, IE{});
                     else
                         exps(std::integral_constant<int, C::EX2_EMU>{}, IH{}, IE{});
+                    if (need_mask) fix_masked(IH{}, IE{});
                     tmem_st32(p_base + BN / 4, *reinterpret_cast<uint32_t(*)[32]>(&pk[BN / 4]));
                     const float2 ps01 = fadd2(ps[0], ps[1]);
                     const float2 ps23 = fadd2(ps[2], ps[3]);
@@ -922,6 +951,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     exps(I0{}, I0{}, IE{});
                 else
                     exps(std::integral_constant<int, C::EX2_EMU>{}, I0{}, IE{});
+                if (need_mask) fix_masked(I0{}, IE{});
                 if constexpr (C::SPLIT_P) {
                     // P_s(j) reuses P_s(j-1)'s columns and O_s is about to be
                     // rescaled: PV_s(j-1) must be complete. (The first step of

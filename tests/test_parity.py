@@ -152,6 +152,37 @@ def test_window_zero_returns_values_exactly(attn, d):
     assert (lse.double().cpu() - ref).abs().max() <= 1e-3
 
 
+def _allowed(i, j, n, causal, window, block):
+    """Key j is attended by query i (the mask's plain definition)."""
+    if block > 0:
+        lo, hi = max(0, (i // block - 1) * block), (i if causal else min(n - 1, (i // block + 1) * block - 1))
+    else:
+        lo = max(0, i - window) if window >= 0 else 0
+        hi = i if causal else (min(n - 1, i + window) if window >= 0 else n - 1)
+    return lo <= j <= hi
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal,window,block,J", [(True, -1, 0, [200, 250, 299]), (True, 100, 0, [5, 130, 299]),
+                                                   (False, 100, 0, [5, 299]), (True, -1, 96, [20, 250])])
+def test_masked_keys_carry_exactly_zero_weight(attn, schedule, d, causal, window, block, J):
+    """A masked key reaches no output: with V at the keys J set to the largest
+    finite bf16 value, every row that attends none of J gives the same bits
+    as before (a weight of even 2^-125 on a masked key would show), and LSE
+    does not change at all."""
+    n = 300
+    q, k, v = synth.make_qkv(1, 2, n, d, seed=36, q_std=4.0)
+    v2 = v.clone()
+    v2[..., J, :] = torch.finfo(torch.bfloat16).max
+    o1, l1 = attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), None, causal, window, block=block)
+    o2, l2 = attn.attn_fwd(q.cuda(), k.cuda(), v2.cuda(), None, causal, window, block=block)
+    assert attn.sync_status() == attn.ATTN_OK
+    rows = [i for i in range(n) if not any(_allowed(i, j, n, causal, window, block) for j in J)]
+    assert len(rows) > 50
+    assert torch.equal(o1[..., rows, :], o2[..., rows, :])
+    assert torch.equal(l1, l2)
+
+
 def test_key_value_permutation_invariance(attn):
     q, k, v = synth.make_qkv(1, 2, 512, 128, seed=32, q_std=4.0)
     perm = torch.randperm(512, generator=torch.Generator().manual_seed(1))
