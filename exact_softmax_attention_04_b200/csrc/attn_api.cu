@@ -92,7 +92,7 @@ namespace {
 
 using namespace attn_host;
 
-bool g_smem_set[kMaxDevices][2][2][2] = {};  // [device][d==128][block mask][persistent]
+bool g_smem_set[kMaxDevices][2][2][2][2] = {};  // [device][d==128][block mask][persistent][no mask]
 int g_num_sms[kMaxDevices] = {};
 
 struct Staging {
@@ -166,12 +166,12 @@ int check_args(const void *q, const void *k, const void *v, const void *o, const
 
 // Sets the kernel's launch attributes once per device and checks its
 // register count against the split it was compiled for.
-template <int D, bool BLOCKMASK, bool PERSIST>
+template <int D, bool BLOCKMASK, bool PERSIST, bool NOMASK>
 int prepare_fwd(int dev)
 {
     using Cfg = attn_sm100::FwdCfg<D>;
     std::lock_guard<std::mutex> lk(g_mu);
-    bool &set = g_smem_set[dev][D == 128 ? 1 : 0][BLOCKMASK ? 1 : 0][PERSIST ? 1 : 0];
+    bool &set = g_smem_set[dev][D == 128 ? 1 : 0][BLOCKMASK ? 1 : 0][PERSIST ? 1 : 0][NOMASK ? 1 : 0];
     if (set) return ATTN_OK;
     if (!g_num_sms[dev] &&
         (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -182,10 +182,10 @@ int prepare_fwd(int dev)
     // computed for (else the raising warps wait forever). Refuse to launch a
     // build that differs.
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST>) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST, NOMASK>) != cudaSuccess)
         return ATTN_ERR_CUDA;
     if (fa.numRegs != static_cast<int>(Cfg::REGS_LAUNCH)) return ATTN_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST>,
+    if (cudaFuncSetAttribute(attn_sm100::attn_fwd_kernel<D, BLOCKMASK, PERSIST, NOMASK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess)
         return ATTN_ERR_CUDA;
@@ -269,22 +269,31 @@ int launch_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
     const FwdSchedule sched = fwd_schedule(n, causal, p.window, p.block);
     const bool persist = sched != kPerItem;
     p.pair_major = sched == kPersistPairMajor ? 1 : 0;
+    // No mask and whole key tiles: no tile is ever masked, so the build
+    // without the mask code runs it.
+    const bool nomask = !blockmask && !causal && p.window < 0 && n % attn_sm100::BN == 0;
     int prc = ATTN_OK;
     if (blockmask)
-        prc = persist ? prepare_fwd<D, true, true>(dev) : prepare_fwd<D, true, false>(dev);
+        prc = persist ? prepare_fwd<D, true, true, false>(dev) : prepare_fwd<D, true, false, false>(dev);
+    else if (nomask)
+        prc = persist ? prepare_fwd<D, false, true, true>(dev) : prepare_fwd<D, false, false, true>(dev);
     else
-        prc = persist ? prepare_fwd<D, false, true>(dev) : prepare_fwd<D, false, false>(dev);
+        prc = persist ? prepare_fwd<D, false, true, false>(dev) : prepare_fwd<D, false, false, false>(dev);
     if (prc != ATTN_OK) return prc;
     const unsigned grid = static_cast<unsigned>(persist ? std::min(p.num_work, g_num_sms[dev]) : p.num_work);
     using namespace attn_sm100;
     if (blockmask && persist)
-        attn_fwd_kernel<D, true, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        attn_fwd_kernel<D, true, true, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     else if (blockmask)
-        attn_fwd_kernel<D, true, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        attn_fwd_kernel<D, true, false, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else if (nomask && persist)
+        attn_fwd_kernel<D, false, true, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+    else if (nomask)
+        attn_fwd_kernel<D, false, false, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     else if (persist)
-        attn_fwd_kernel<D, false, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        attn_fwd_kernel<D, false, true, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     else
-        attn_fwd_kernel<D, false, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+        attn_fwd_kernel<D, false, false, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

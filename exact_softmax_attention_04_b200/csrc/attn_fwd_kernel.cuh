@@ -55,7 +55,10 @@
 // reloads Q_s once the last S_s MMA of the previous item is done (q_empty),
 // the first PV_s of an item waits until the softmax has read the previous
 // O_s out (o_free), and the epilogue writes O straight from registers to
-// global memory (the Q buffer may already hold the next item's Q).
+// global memory (the Q buffer may already hold the next item's Q). NOMASK:
+// compiled without the mask code, for problems with no mask whose length is a
+// whole number of key tiles (no tile is ever masked): the masked branches,
+// never taken there, otherwise still cost 1% to 4% on unmasked rows.
 //
 // Every wait is bounded (about one second). On expiry the kernel sets bit 1
 // of the device status word, tells the other roles to stop, waits (bounded)
@@ -361,7 +364,9 @@ __device__ __forceinline__ int fwd_item(const FwdParams &p, int k)
 // ... (for short key ranges, where a CTA's start-up, Q load and epilogue
 // would otherwise not be amortised); else one CTA per work item. Every
 // mbarrier phase is counted across items, so both forms run the same code.
-template <int D, bool BLOCKMASK, bool PERSIST>
+// NOMASK: no mask and n a multiple of BN (the host chooses it; never with
+// BLOCKMASK).
+template <int D, bool BLOCKMASK, bool PERSIST, bool NOMASK>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -789,12 +794,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                               : ((k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
                                  (!causal && window >= 0 && k0 + BN - 1 > q0 + window));
                 const bool mask_lo = BLOCKMASK ? (tile_first > k0) : (window >= 0 && k0 < q0 + BM - 1 - window);
-                const bool need_mask = mask_hi || mask_lo;
+                const bool need_mask = !NOMASK && (mask_hi || mask_lo);
                 // Allowed keys of this row form one interval; in tile columns:
-                // [col_lo(), col_hi()] with key = k0 + column (on a side that
-                // cuts no row, the bound lies outside the tile). Evaluated
-                // where used: at d = 128 only inside the masked branch (1%
-                // faster on persistent windows than computing them up front).
+                // [lo, hi] with key = k0 + column (on a side that cuts no row,
+                // the bound lies outside the tile). At d = 64 computed up
+                // front (the zeroing after the exponentials needs them too),
+                // at d = 128 inside the masked branch: 1% faster each.
                 auto col_hi = [&]() {
                     return BLOCKMASK ? row_last - k0
                                      : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
@@ -803,10 +808,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 auto col_lo = [&]() {
                     return BLOCKMASK ? row_first - k0 : ((window >= 0) ? row - window - k0 : 0);
                 };
+                int hi = 0, lo = 0;
+                if constexpr (C::EMU_MASKED) {
+                    hi = col_hi();
+                    lo = col_lo();
+                }
                 if (need_mask) {
                     // Most masked tiles cut on one side only, which takes one
                     // compare per element.
-                    const int hi = col_hi(), lo = col_lo();
+                    if constexpr (!C::EMU_MASKED) {
+                        hi = col_hi();
+                        lo = col_lo();
+                    }
                     if (mask_hi && mask_lo) {
 #pragma unroll
                         for (int c = 0; c < BN; ++c)
@@ -898,7 +911,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // before that is scaled away by alpha = 0).
                 auto fix_masked = [&](auto i0, auto i1) {
                     if constexpr (C::EMU_MASKED && C::EX2_EMU > 0) {
-                        const int hi = col_hi(), lo = col_lo();
 #pragma unroll
                         for (int i = decltype(i0)::value; i < decltype(i1)::value; ++i) {
                             if ((C::EMU_SPREAD ? ((i * C::EX2_EMU) % 16) : (i % 16)) < C::EX2_EMU) {
