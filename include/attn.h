@@ -31,7 +31,8 @@
  *                              local attention section of the same page)
  * A window of n - 1 or more allows the same keys as no window. The
  * block-local mask has entry points of its own (attn_fwd_blocklocal,
- * attn_bwd_blocklocal).
+ * attn_bwd_blocklocal). A key the mask excludes gets a weight of exactly 0:
+ * its values never reach O, whatever they are (finite).
  *
  * Layout: Q, K, V and O are bf16, contiguous [B, H, n, d] (token-major inside
  * each head, d fastest). LSE is fp32, contiguous [B, H, n], natural-log units.
