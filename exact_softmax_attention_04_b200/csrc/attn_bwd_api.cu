@@ -18,6 +18,7 @@ namespace {
 using namespace attn_host;
 
 bool g_bwd_set[kMaxDevices][2][2] = {};  // [device][d==128][general]
+bool g_bwd_nomask_set[kMaxDevices][2] = {};  // fused kernel without mask code: [device][d==128]
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -192,14 +193,23 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
         !encode_bhnd(enc, &mdk, dk, bhkv, n, D) || !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
     const bool general = effective_block(n, block) > 0 || Hkv != H;
+    // No mask and whole tiles: no tile needs a mask, the build without the
+    // mask test runs it.
+    const bool nomask = !general && !causal && effective_window(n, window) < 0 && n % attn_sm100::BN == 0;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
+        bool &set = nomask ? g_bwd_nomask_set[dev][D == 128 ? 1 : 0] : g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
         if (!set) {
-            const int rc =
-                general
-                    ? prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, true>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH)
-                    : prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, false>, Cfg::SMEM_BYTES, Cfg::REGS_LAUNCH);
+            int rc;
+            if (general)
+                rc = prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, true, false>, Cfg::SMEM_BYTES,
+                                    Cfg::REGS_LAUNCH);
+            else if (nomask)
+                rc = prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, false, true>, Cfg::SMEM_BYTES,
+                                    Cfg::REGS_LAUNCH);
+            else
+                rc = prepare_kernel(attn_sm100::attn_bwd_fused_kernel<D, false, false>, Cfg::SMEM_BYTES,
+                                    Cfg::REGS_LAUNCH);
             if (rc != ATTN_OK) return rc;
             set = true;
         }
@@ -236,10 +246,13 @@ int launch_bwd_fused(const void *q, const void *k, const void *v, const void *o,
     p.block = effective_block(n, block);
     const unsigned grid = static_cast<unsigned>(bhkv * p.num_k_tiles);
     if (general)
-        attn_sm100::attn_bwd_fused_kernel<D, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_fused_kernel<D, true, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, macc, p);
+    else if (nomask)
+        attn_sm100::attn_bwd_fused_kernel<D, false, true><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdk, mdv, macc, p);
     else
-        attn_sm100::attn_bwd_fused_kernel<D, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_fused_kernel<D, false, false><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdk, mdv, macc, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
