@@ -18,7 +18,7 @@ namespace {
 using namespace attn_host;
 
 bool g_bwd_set[kMaxDevices][2][2] = {};  // [device][d==128][general]
-bool g_bwd_nomask_set[kMaxDevices][2] = {};  // fused kernel without mask code: [device][d==128]
+bool g_bwd_nomask_set[kMaxDevices][2] = {};  // kernels without mask code: [device][d==128]
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -108,17 +108,26 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
         !encode_bhnd(enc, &mdv, dv, bhkv, n, D))
         return ATTN_ERR_CUDA;
     const bool general = effective_block(n, block) > 0 || Hkv != H;
+    // No mask and whole tiles: the builds without the mask test run it.
+    const bool nomask = !general && !causal && effective_window(n, window) < 0 && n % attn_sm100::BN == 0;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        bool &set = g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
+        bool &set = nomask ? g_bwd_nomask_set[dev][D == 128 ? 1 : 0] : g_bwd_set[dev][D == 128 ? 1 : 0][general ? 1 : 0];
         if (!set) {
-            int rc = general
-                         ? prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, true>, KV::SMEM_BYTES, KV::REGS_LAUNCH)
-                         : prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, false>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
-            if (rc == ATTN_OK)
-                rc = general
-                         ? prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, true>, QC::SMEM_BYTES, QC::REGS_LAUNCH)
-                         : prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, false>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+            int rc;
+            if (general) {
+                rc = prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, true, false>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
+                if (rc == ATTN_OK)
+                    rc = prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, true, false>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+            } else if (nomask) {
+                rc = prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, false, true>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
+                if (rc == ATTN_OK)
+                    rc = prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, false, true>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+            } else {
+                rc = prepare_kernel(attn_sm100::attn_bwd_dkdv_kernel<D, false, false>, KV::SMEM_BYTES, KV::REGS_LAUNCH);
+                if (rc == ATTN_OK)
+                    rc = prepare_kernel(attn_sm100::attn_bwd_dq_kernel<D, false, false>, QC::SMEM_BYTES, QC::REGS_LAUNCH);
+            }
             if (rc != ATTN_OK) return rc;
             set = true;
         }
@@ -156,20 +165,26 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *o, const
     // 2. dK, dV: one CTA per key tile of each key/value head
     const unsigned kv_grid = static_cast<unsigned>(bhkv * p.num_k_tiles);
     if (general)
-        attn_sm100::attn_bwd_dkdv_kernel<D, true><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_dkdv_kernel<D, true, false><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdk, mdv, p);
+    else if (nomask)
+        attn_sm100::attn_bwd_dkdv_kernel<D, false, true><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdk, mdv, p);
     else
-        attn_sm100::attn_bwd_dkdv_kernel<D, false><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_dkdv_kernel<D, false, false><<<kv_grid, KV::THREADS, KV::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdk, mdv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
     // 3. dQ: one CTA per query tile
     const unsigned q_grid = static_cast<unsigned>(bh * p.num_q_tiles);
     if (general)
-        attn_sm100::attn_bwd_dq_kernel<D, true><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_dq_kernel<D, true, false><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdq, p);
+    else if (nomask)
+        attn_sm100::attn_bwd_dq_kernel<D, false, true><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdq, p);
     else
-        attn_sm100::attn_bwd_dq_kernel<D, false><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
+        attn_sm100::attn_bwd_dq_kernel<D, false, false><<<q_grid, QC::THREADS, QC::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdq, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

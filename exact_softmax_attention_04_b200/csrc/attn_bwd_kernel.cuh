@@ -282,8 +282,11 @@ __device__ __forceinline__ bool smem_base_1k(uint8_t *raw_ptr, uint32_t &base, u
 // ---------------------------------------------------------------------------
 // 2. dK and dV. GENERAL: compiled for grouped-query heads (kv_heads <
 // heads) or the block-local mask (block > 0); the other instantiation handles
-// multi-head attention under the causal and window masks.
-template <int D, bool GENERAL>
+// multi-head attention under the causal and window masks. NOMASK (never with
+// GENERAL): compiled without the mask test, for problems with no mask whose
+// length is a whole number of tiles (no tile needs one; the test, never
+// taken there, still cost 2%).
+template <int D, bool GENERAL, bool NOMASK>
 __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -520,9 +523,9 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
                 lo = key_first - q0;
                 hi = (key < n) ? key_last - q0 : -1;
             } else {
-                need_mask = (k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
-                            (window >= 0 && q0 + BM - 1 > k0 + window) ||
-                            (!causal && window >= 0 && q0 < k0 + BN - 1 - window);
+                need_mask = !NOMASK && ((k0 + BN > n) || (q0 + BM > n) || (causal && q0 < k0 + BN - 1) ||
+                                        (window >= 0 && q0 + BM - 1 > k0 + window) ||
+                                        (!causal && window >= 0 && q0 < k0 + BN - 1 - window));
                 lo = causal ? key - q0 : (window >= 0 ? key - window - q0 : 0);
                 hi = min(BM - 1, n - 1 - q0);
                 if (window >= 0) hi = min(hi, key + window - q0);
@@ -637,9 +640,9 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
 
 // ---------------------------------------------------------------------------
 // 3. dQ.
-// GENERAL as for attn_bwd_dkdv_kernel (here only the mask arithmetic
-// differs: the head mapping is the same for both).
-template <int D, bool GENERAL>
+// GENERAL and NOMASK as for attn_bwd_dkdv_kernel (here only the mask
+// arithmetic differs: the head mapping is the same for both).
+template <int D, bool GENERAL, bool NOMASK>
 __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -870,10 +873,10 @@ __global__ void __launch_bounds__(BwdRoles::THREADS, 1)
             tc_fence_before();
             mbar_arrive(s_read);
             const bool need_mask =
-                GENERAL ? ((k0 + BN > n) || tile_first > k0 || tile_last < k0 + BN - 1)
-                          : ((k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
-                             (window >= 0 && k0 < q0 + BM - 1 - window) ||
-                             (!causal && window >= 0 && k0 + BN - 1 > q0 + window));
+                !NOMASK && (GENERAL ? ((k0 + BN > n) || tile_first > k0 || tile_last < k0 + BN - 1)
+                                    : ((k0 + BN > n) || (causal && k0 + BN - 1 > q0) ||
+                                       (window >= 0 && k0 < q0 + BM - 1 - window) ||
+                                       (!causal && window >= 0 && k0 + BN - 1 > q0 + window)));
             // allowed key columns of this row: [lo, hi], key = k0 + column
             const int hi = GENERAL ? row_last - k0
                                      : min(causal ? row - k0 : (window >= 0 ? row + window - k0 : BN - 1),
