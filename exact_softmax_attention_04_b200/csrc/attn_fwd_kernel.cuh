@@ -20,10 +20,11 @@
 //              masks boundary tiles, updates (m, l), writes P (bf16) into TMEM,
 //              rescales its O row when m grew, and runs the epilogue
 //              (O / l -> bf16 -> smem -> TMA store; LSE store).
-//   warp 8     MMA issuer (one elected lane) and TMEM owner.
+//   warp 8     MMA issuer (one elected lane) and TMEM owner; in the
+//              persistent form it issues Q_0's MMAs and warp 10 Q_1's.
 //   warp 9     TMA producer (one elected lane): Q_0, Q_1 once, then K_j, V_j
 //              alternately into a ring of NSLOT shared-memory slots.
-//   warps 10-11 idle (they complete the third warpgroup).
+//   warps 10-11 otherwise idle (they complete the third warpgroup).
 // Registers: launched at 168 per thread; the softmax warpgroups raise theirs
 // to 232 (a 128-float S row plus its P stay in registers, no spills) and the
 // third warpgroup drops to 40: 2*128*232 + 128*40 = 384*168.
@@ -35,9 +36,9 @@
 // overwrites P_s(j-1) only after PV_s(j-1) has read it, and (b) when S_s(j)
 // is complete, PV_s(j-1) is too, so the softmax may rescale O_s right away.
 // With one CTA per item the softmax hands P_s over in two halves (keys 0..63,
-// then 64..127, each announced on its own barrier, O_s rescaled before the
-// first): the MMA warp issues PV_s on the first half while the softmax is
-// still computing the second.
+// then 64..127, each announced on its own barrier; O_s is rescaled before the
+// first is announced): the MMA warp issues PV_s on the first half while the
+// softmax is still computing the second.
 // D = 64: S_0(j), S_1(j), PV_0(j-1), PV_1(j-1), S_s(j) waiting only until the
 // softmax has read S_s(j-1) into registers; the softmax waits for PV_s(j-1)
 // before it overwrites P_s or rescales O_s.
